@@ -1,0 +1,369 @@
+#!/usr/bin/env python
+"""Benchmark of the linear-logp operator on B200.
+
+One step = the whole hot path on one batch: the forward (fused LM-head GEMM
++ online logsumexp / entropy + target gather, then the fixed-order combine)
+and the backward (per vocab chunk: logits recompute + dlogits, dHidden GEMM,
+dW GEMM).  Default workload: the RL actor step, 8 ragged sequences
+concatenated (T = 5980 for seed 3), H=4096, V=151936, bf16, tau = 1.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU, weak scaling: every rank
+processes its own batch against the same (replicated) W; there is no
+data-path collective (rows are independent).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "linear-logp fwd+bwd tokens/s at H4096 V151936 bf16; % of BF16 TC peak"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % index)
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+        return False
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        except OSError:
+            return None
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def rl_inputs(rank):
+    from invariant_lm_head_gemm_b200 import workloads as wl
+    w = wl.rl_step(3 + 1000 * rank, with_weight=False)
+    W = wl.make_weight(3, wl.QWEN_V, wl.QWEN_H)
+    return w, W
+
+
+def cpu_baseline(w, W, rows=8):
+    """The fp64 oracle, as it stands, on a bounded sample of rows of the same
+    workload (forward + backward), on this host's cores."""
+    import oracle
+    oracle.build()
+    idx = np.linspace(0, w.T - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.forward(w.hidden[idx], W, w.targets[idx], w.temperature)
+    oracle.backward(w.hidden[idx], W, w.targets[idx], w.temperature, w.dlogp[idx],
+                    w.dentropy[idx])
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d of %d rows of the RL actor step (H=4096, V=151936), fp64 C oracle "
+                      "forward + backward, %.1f s" % (rows, w.T, dt)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w, W = rl_inputs(0)
+    import oracle
+    oracle.build()
+    rows_per_step = args.ref_rows
+    rng = np.random.default_rng(0)
+
+    def step():
+        idx = np.sort(rng.choice(w.T, rows_per_step, replace=False))
+        oracle.forward(w.hidden[idx], W, w.targets[idx], w.temperature)
+        oracle.backward(w.hidden[idx], W, w.targets[idx], w.temperature, w.dlogp[idx],
+                        w.dentropy[idx])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = rows_per_step * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Gaussian, bf16-rounded)",
+        "config": config_dict(w, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": "%d random rows of the RL actor step per step "
+                                   "(fwd + bwd, fp64 C oracle)" % rows_per_step},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, world):
+    return {"workload": "rl_actor_step: 8 ragged sequences (lengths U[256,1024], seed 3), "
+                        "fwd+bwd, H=4096, V=151936, bf16, tau=1",
+            "T_per_rank": int(w.T), "H": 4096, "V": 151936, "temperature": 1.0,
+            "seq_lens": [int(x) for x in w.seq_lens], "parallelism": "dp%d" % world,
+            "l2": "inputs larger than L2: all of W (1.245 GB) is read every step"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from invariant_lm_head_gemm_b200 import binding
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w, W_host = rl_inputs(rank)
+    T, H, V = w.T, w.H, w.V
+
+    def to_dev_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    W = to_dev_bf16(W_host)
+    hid = to_dev_bf16(w.hidden)
+    tg = torch.from_numpy(w.targets).to(dev)
+    dl = torch.from_numpy(w.dlogp).to(dev)
+    de = torch.from_numpy(w.dentropy).to(dev)
+    ws = binding.make_workspace(T, H, V, True, dev)
+    logp = torch.empty(T, device=dev)
+    ent = torch.empty(T, device=dev)
+    lse = torch.empty(T, device=dev)
+    dH = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    dW = torch.empty(V, H, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
+        binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent, dl, de, ws, out=(dH, dW))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------------------------------------------------------- device-resident
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    flags = binding.rlk_read_device_error(ws)
+
+    # ---------------------------------------------------------------- forward kernel alone
+    fe0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    fe1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for _ in range(3):
+        binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
+    for i in range(args.steps):
+        fe0[i].record(stream)
+        binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
+        fe1[i].record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(fe0, fe1))
+
+    # ---------------------------------------------------------------- end to end, host buffers
+    hid_h = torch.from_numpy(w.hidden.view(np.int16)).view(torch.bfloat16).pin_memory()
+    tg_h = torch.from_numpy(w.targets).pin_memory()
+    dl_h = torch.from_numpy(w.dlogp).pin_memory()
+    de_h = torch.from_numpy(w.dentropy).pin_memory()
+    out_h = torch.empty(2, T, dtype=torch.float32).pin_memory()
+    res = torch.empty(2, T, dtype=torch.float32, device=dev)
+
+    def e2e_step():
+        hid.copy_(hid_h, non_blocking=True)
+        tg.copy_(tg_h, non_blocking=True)
+        dl.copy_(dl_h, non_blocking=True)
+        de.copy_(de_h, non_blocking=True)
+        binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(res[0], res[1], lse))
+        binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, res[1], dl, de, ws, out=(dH, dW))
+        out_h.copy_(res, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    ee0 = torch.cuda.Event(enable_timing=True)
+    ee1 = torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ee1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = ee0.elapsed_time(ee1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = T * H * 2 + T * 8 + T * 4 + T * 4
+    d2h = 2 * T * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, W_host, rows=args.cpu_rows)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    pk, src = peaks()
+    flops_tok = 8.0 * H * V
+    step_tflops = flops_tok * T / (ms_max * 1e-3) / 1e12
+    fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
+    nchunks = -(-V // 8192)
+    launches_per_step = 2 + 3 * nchunks
+    value = world * T / (ms_max * 1e-3)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian, bf16-rounded; stands in for Qwen3-8B hidden "
+                "states / LM head and DAPO-Math-17k rollouts)",
+        "config": config_dict(w, world),
+        "tflops_per_gpu": step_tflops,
+        "pct_of_bf16_peak": {"burst": step_tflops / pk["bf16_tflops"],
+                             "sustained": step_tflops / pk["bf16_tflops_sustained"],
+                             "datasheet_2250": step_tflops / 2250.0, "peaks": src},
+        "roofline": {"kernel": "forward: fused LM-head GEMM + online logsumexp/entropy "
+                               "+ target gather (+ combine), timed alone",
+                     "bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": fwd_tflops / pk["bf16_tflops"],
+                     "traffic": None, "peak_source": src + " burst bf16",
+                     "flops_per_launch": 2.0 * T * H * V, "ms_per_launch": fwd_ms},
+        "step_roofline": {"bound": "tensor", "achieved": step_tflops,
+                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                          "frac": step_tflops / pk["bf16_tflops_sustained"],
+                          "flops_per_token": flops_tok, "peak_source": src + " sustained bf16"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "device_error_flags": flags,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=48)
+    ap.add_argument("--ref-rows", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,145 @@
+/*
+ * rlk.h -- C ABI of librlk: the bitwise batch-invariant linear-logp operator
+ * (LM head GEMM -> temperature -> full-vocab logsumexp, target log-prob and
+ * entropy, plus its backward to dHidden and dW) for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  The RL-Kernel pages name a linear-logp route,
+ * "rlkernel.linear_logp.bitwise.v1" (h100-cp-gradient.json,
+ * runs[].validation.runtime_readbacks.frameworks.{megatron/training,
+ * vllm/rollout}.modules.logp), that stands in for VIME's native
+ * calculate_log_probs_and_entropy (VIME Qwen3-8B TP4/CP2 dense page,
+ * "User-facing operator matrix") and whose train and rollout results must be
+ * bitwise equal (same page, "Required gates": zero bitwise mismatches, no
+ * fallback; h100-cp-gradient.json runs[0].validation.train_rollout_logprob:
+ * bitwise_equal, 0 mismatches over 8192 elements).  The pages print no
+ * formula; this library computes, for each row t and the whole vocabulary,
+ *
+ *   z[t,v]     = (sum_h hidden[t,h] * W[v,h]) / temperature
+ *   lse[t]     = log sum_v exp(z[t,v])
+ *   logp[t]    = z[t,targets[t]] - lse[t]
+ *   entropy[t] = lse[t] - sum_v p[t,v] z[t,v],       p = exp(z - lse)
+ *
+ * and, given upstream gradients dlogp[t] and dentropy[t],
+ *
+ *   dx[t,v]      = (dlogp[t] (1[v = targets[t]] - p[t,v])
+ *                   - dentropy[t] p[t,v] (z[t,v] - (lse[t] - entropy[t]))) / temperature
+ *   dHidden[t,:] = sum_v dx[t,v] W[v,:]
+ *   dW[v,:]      = sum_t dx[t,v] hidden[t,:]
+ *
+ * The T x V logits are never written to memory.
+ *
+ * Determinism contract.  For a given (H, V, temperature), every per-row output
+ * (logp, entropy, lse and the dHidden row) depends only on that row's hidden
+ * vector, target and gradient seeds: it is bitwise the same for any T, any
+ * position of the row in the batch and any other rows in the batch, and
+ * bitwise the same run to run.  dW (a sum over rows) is bitwise repeatable
+ * for identical inputs: fixed summation order, no atomics.
+ *
+ * Conventions for every entry point below.
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *    contiguous.  bf16 tensors are passed as rlk_bf16 (the raw 16-bit
+ *    pattern).  hidden, W, dHidden and dW must be 16-byte aligned, the
+ *    workspace 256-byte aligned; the float and int64 vectors need their
+ *    natural alignment.
+ *  - The library allocates no memory and keeps no per-call state; everything
+ *    is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *    with no host synchronisation.  Kernel launch parameters are fixed at
+ *    enqueue time, so a call can be captured into a CUDA graph.
+ *  - Errors are fail-closed: bad arguments are rejected with a status before
+ *    anything is enqueued and there is no fallback route of any kind.
+ *  - Supported shapes: 64 <= H <= 2^20, H % 64 == 0; 1 <= V < 2^31;
+ *    0 <= T < 2^31.
+ *    T == 0 is a successful no-op (bwd still zeroes dW).
+ *  - Device faults are reported, never trapped: a target outside [0, V)
+ *    yields NaN logp for that row (its dHidden row omits the one-hot term)
+ *    and sets RLK_DEVERR_TARGET in the workspace's error word; an internal
+ *    pipeline wait that exceeds its time bound sets RLK_DEVERR_TIMEOUT and
+ *    the kernel exits.  Read (and clear) the word with
+ *    rlk_read_device_error.
+ */
+#ifndef RLK_H_
+#define RLK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t rlk_bf16;
+
+typedef enum {
+  RLK_OK = 0,
+  RLK_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad temperature */
+  RLK_ERR_UNSUPPORTED_SHAPE = 2,  /* H % 64 != 0, sizes out of range            */
+  RLK_ERR_MISALIGNED = 3,         /* pointer alignment below the stated minimum  */
+  RLK_ERR_WORKSPACE_TOO_SMALL = 4,
+  RLK_ERR_UNSUPPORTED_DEVICE = 5, /* current device is not compute capability 10.0 */
+  RLK_ERR_CUDA = 6                /* a CUDA runtime/driver call or launch failed */
+} rlk_status;
+
+/* Bits of the device error word at the start of the workspace. */
+#define RLK_DEVERR_TARGET 0x1u
+#define RLK_DEVERR_TIMEOUT 0x2u
+
+/* Bytes of workspace that rlk_linear_logp_fwd (for_backward == 0) or both
+ * rlk_linear_logp_fwd and rlk_linear_logp_bwd (for_backward != 0) need for
+ * these sizes.  Returns 0 for unsupported sizes.  The first 256 bytes hold
+ * the device error word: zero them once when the workspace is allocated (or
+ * call rlk_read_device_error once); the library never clears it on its own. */
+size_t rlk_linear_logp_workspace_bytes(int64_t T, int64_t H, int64_t V, int for_backward);
+
+/* Forward.  hidden [T,H] bf16, W [V,H] bf16 (the LM head, one row per vocab
+ * entry), targets [T] int64 in [0, V), temperature > 0 and finite.  Writes
+ * logp, entropy and lse, each [T] fp32 (natural log, lse of the temperature-
+ * scaled logits).  Uses the workspace for per-(row, vocab split) partials. */
+rlk_status rlk_linear_logp_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                               int64_t T, int64_t H, int64_t V, float temperature, float* logp,
+                               float* entropy, float* lse, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Backward.  Same hidden, W, targets, sizes and temperature as the forward;
+ * lse and entropy are the forward's outputs for these rows; dlogp and
+ * dentropy [T] fp32 are the upstream gradients of logp and entropy.
+ * Overwrites dHidden [T,H] bf16 and dW [V,H] fp32 (no accumulation into
+ * existing contents).  The logits are recomputed one vocab chunk at a time;
+ * the chunk's dlogits are rounded to bf16 in the workspace before the two
+ * gradient GEMMs. */
+rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                               int64_t T, int64_t H, int64_t V, float temperature,
+                               const float* lse, const float* entropy, const float* dlogp,
+                               const float* dentropy, rlk_bf16* dHidden, float* dW,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Self-check of the tensor-core mainloop shared by every kernel above:
+ * C[M,N] fp32 = sum_k A[m,k] B[n,k] with bf16 inputs and fp32 accumulation.
+ * a_mn_major == 0: A is stored [M,K] (K contiguous); != 0: stored [K,M].
+ * b_mn_major == 0: B is stored [N,K]; != 0: stored [K,N].  M, N, K >= 1 and
+ * multiples of 8.  Not part of the operator; the pages have no counterpart.
+ * Needs a workspace of rlk_gemm_workspace_bytes() bytes for its error word. */
+size_t rlk_gemm_workspace_bytes(void);
+rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, int64_t N,
+                             int64_t K, int a_mn_major, int b_mn_major, float* C,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Provenance readback, in the spirit of the pages' per-module runtime
+ * readbacks (h100-cp-gradient.json, runs[].validation.runtime_readbacks:
+ * backend_ids, call_count).  rlk_backend_id() names this implementation;
+ * rlk_call_count(0) / (1) / (2) count successfully enqueued forward /
+ * backward / self-check GEMM calls in this process. */
+const char* rlk_backend_id(void);
+uint64_t rlk_call_count(int which);
+
+/* Copies the device error word (RLK_DEVERR_* bits) of `workspace` to *flags,
+ * then clears it.  Synchronises `stream`. */
+rlk_status rlk_read_device_error(void* workspace, uint32_t* flags, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* rlk_status_string(rlk_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RLK_H_ */

@@ -1,0 +1,209 @@
+"""Thin Python binding of librlk.so (include/rlk.h) for torch tensors.
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels.  There is no fallback; if the library is missing or the device
+is not a B200 the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librlk.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "rlk.h")
+
+RLK_DEVERR_TARGET = 0x1
+RLK_DEVERR_TIMEOUT = 0x2
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_lib = None
+
+
+class RlkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s" % (what, status_string(status)))
+
+
+def lib():
+    """Load librlk.so (built in-tree by ``python -m invariant_lm_head_gemm_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("librlk.so is not built (%s); run "
+                               "`python -m invariant_lm_head_gemm_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        L.rlk_linear_logp_workspace_bytes.argtypes = [_I64, _I64, _I64, ctypes.c_int]
+        L.rlk_linear_logp_workspace_bytes.restype = ctypes.c_size_t
+        L.rlk_linear_logp_fwd.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float,
+                                          _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.rlk_linear_logp_fwd.restype = ctypes.c_int
+        L.rlk_linear_logp_bwd.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float,
+                                          _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.rlk_linear_logp_bwd.restype = ctypes.c_int
+        L.rlk_gemm_workspace_bytes.argtypes = []
+        L.rlk_gemm_workspace_bytes.restype = ctypes.c_size_t
+        L.rlk_gemm_bf16_f32.argtypes = [_P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                        _P, _P, ctypes.c_size_t, _P]
+        L.rlk_gemm_bf16_f32.restype = ctypes.c_int
+        L.rlk_backend_id.argtypes = []
+        L.rlk_backend_id.restype = ctypes.c_char_p
+        L.rlk_call_count.argtypes = [ctypes.c_int]
+        L.rlk_call_count.restype = ctypes.c_uint64
+        L.rlk_read_device_error.argtypes = [_P, ctypes.POINTER(ctypes.c_uint32), _P]
+        L.rlk_read_device_error.restype = ctypes.c_int
+        L.rlk_status_string.argtypes = [ctypes.c_int]
+        L.rlk_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def declared_functions():
+    """Names of the functions declared in include/rlk.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rlk_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return lib().rlk_status_string(int(status)).decode()
+
+
+def backend_id() -> str:
+    return lib().rlk_backend_id().decode()
+
+
+def call_count(which: int) -> int:
+    return int(lib().rlk_call_count(which))
+
+
+def _check(status, what):
+    if status != 0:
+        raise RlkError(status, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_bytes(T: int, H: int, V: int, for_backward: bool = True) -> int:
+    return int(lib().rlk_linear_logp_workspace_bytes(T, H, V, 1 if for_backward else 0))
+
+
+def make_workspace(T: int, H: int, V: int, for_backward: bool = True, device=None):
+    """A zeroed workspace tensor (uint8) big enough for these sizes."""
+    n = workspace_bytes(T, H, V, for_backward)
+    if n == 0:
+        raise ValueError("unsupported sizes T=%d H=%d V=%d" % (T, H, V))
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _req(t, dtype, name, ndim):
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous() or t.dim() != ndim:
+        raise ValueError("%s must be a contiguous CUDA %s tensor with %d dims" % (name, dtype, ndim))
+
+
+def rlk_linear_logp_fwd(hidden, W, targets, temperature, workspace=None, out=None, stream=None):
+    """logp, entropy, lse [T] fp32 of hidden [T,H] bf16 against W [V,H] bf16."""
+    _req(hidden, torch.bfloat16, "hidden", 2)
+    _req(W, torch.bfloat16, "W", 2)
+    _req(targets, torch.int64, "targets", 1)
+    T, H = hidden.shape
+    V = W.shape[0]
+    if W.shape[1] != H or targets.shape[0] != T:
+        raise ValueError("shape mismatch")
+    if workspace is None:
+        workspace = make_workspace(T, H, V, False, hidden.device)
+    if out is None:
+        out = tuple(torch.empty(T, dtype=torch.float32, device=hidden.device) for _ in range(3))
+    logp, entropy, lse = out
+    _check(lib().rlk_linear_logp_fwd(_ptr(hidden), _ptr(W), _ptr(targets), T, H, V,
+                                     float(temperature), _ptr(logp), _ptr(entropy), _ptr(lse),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+           "rlk_linear_logp_fwd")
+    return logp, entropy, lse
+
+
+def rlk_linear_logp_bwd(hidden, W, targets, temperature, lse, entropy, dlogp, dentropy,
+                        workspace=None, out=None, stream=None):
+    """dHidden [T,H] bf16 and dW [V,H] fp32 (both overwritten)."""
+    _req(hidden, torch.bfloat16, "hidden", 2)
+    _req(W, torch.bfloat16, "W", 2)
+    _req(targets, torch.int64, "targets", 1)
+    for n, t in (("lse", lse), ("entropy", entropy), ("dlogp", dlogp), ("dentropy", dentropy)):
+        _req(t, torch.float32, n, 1)
+    T, H = hidden.shape
+    V = W.shape[0]
+    if workspace is None:
+        workspace = make_workspace(T, H, V, True, hidden.device)
+    if out is None:
+        out = (torch.empty(T, H, dtype=torch.bfloat16, device=hidden.device),
+               torch.empty(V, H, dtype=torch.float32, device=hidden.device))
+    dHidden, dW = out
+    _check(lib().rlk_linear_logp_bwd(_ptr(hidden), _ptr(W), _ptr(targets), T, H, V,
+                                     float(temperature), _ptr(lse), _ptr(entropy), _ptr(dlogp),
+                                     _ptr(dentropy), _ptr(dHidden), _ptr(dW), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)),
+           "rlk_linear_logp_bwd")
+    return dHidden, dW
+
+
+def rlk_gemm_bf16_f32(A, B, a_mn_major=False, b_mn_major=False, stream=None):
+    """C = A' . B'^T through the tensor-core mainloop (self-check entry).
+    A' is A ([M,K]) or A^T (A stored [K,M] when a_mn_major); B' likewise."""
+    _req(A, torch.bfloat16, "A", 2)
+    _req(B, torch.bfloat16, "B", 2)
+    M, K = (A.shape[1], A.shape[0]) if a_mn_major else A.shape
+    N, K2 = (B.shape[1], B.shape[0]) if b_mn_major else B.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+    ws = torch.zeros(int(lib().rlk_gemm_workspace_bytes()), dtype=torch.uint8, device=A.device)
+    _check(lib().rlk_gemm_bf16_f32(_ptr(A), _ptr(B), M, N, K, int(a_mn_major), int(b_mn_major),
+                                   _ptr(C), _ptr(ws), ws.numel(), _stream(stream)),
+           "rlk_gemm_bf16_f32")
+    return C, ws
+
+
+def rlk_read_device_error(workspace, stream=None) -> int:
+    """RLK_DEVERR_* bits recorded in the workspace (then cleared).  Syncs."""
+    v = ctypes.c_uint32(0)
+    _check(lib().rlk_read_device_error(_ptr(workspace), ctypes.byref(v), _stream(stream)),
+           "rlk_read_device_error")
+    return int(v.value)
+
+
+class LinearLogp(torch.autograd.Function):
+    """autograd wrapper: (logp, entropy) = LinearLogp.apply(hidden, W, targets, temperature).
+    Gradients flow to hidden (bf16) and W (fp32 cast to W's dtype)."""
+
+    @staticmethod
+    def forward(ctx, hidden, W, targets, temperature):
+        T, H = hidden.shape
+        ws = make_workspace(T, H, W.shape[0], True, hidden.device)
+        logp, entropy, lse = rlk_linear_logp_fwd(hidden, W, targets, temperature, ws)
+        ctx.save_for_backward(hidden, W, targets, lse, entropy)
+        ctx.temperature = temperature
+        ctx.ws = ws
+        return logp, entropy
+
+    @staticmethod
+    def backward(ctx, dlogp, dentropy):
+        hidden, W, targets, lse, entropy = ctx.saved_tensors
+        T = hidden.shape[0]
+        dl = (dlogp if dlogp is not None else torch.zeros(T, device=hidden.device)).float()
+        de = (dentropy if dentropy is not None else torch.zeros(T, device=hidden.device)).float()
+        dH, dW = rlk_linear_logp_bwd(hidden, W, targets, ctx.temperature, lse, entropy,
+                                     dl.contiguous(), de.contiguous(), ctx.ws)
+        return dH, dW.to(W.dtype), None, None

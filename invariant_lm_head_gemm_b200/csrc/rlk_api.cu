@@ -1,0 +1,415 @@
+// rlk_api.cu -- the C ABI declared in include/rlk.h: argument checks,
+// workspace layout, TMA tensor-map encoding and the launch sequences of the
+// forward and backward passes.  No allocation, no host synchronisation
+// (except rlk_read_device_error), no fallback path.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "rlk.h"
+#include "rlk_gemm.cuh"
+
+namespace rlk {
+namespace {
+
+// Vocab tiles per forward unit: each (row, split of 2 x 256 vocab entries)
+// yields one online triple.  Fixed, so partials never depend on T.
+constexpr int kFwdGroup = 2;
+// Vocab chunk of the backward: dlogits for kVChunk vocab entries at a time
+// go through the workspace.  Fixed (for a given V), so dHidden rows never
+// depend on T.
+constexpr int64_t kVChunk = 8192;
+constexpr size_t kHeader = 256;  // device error word + padding
+
+std::atomic<uint64_t> g_calls[3];
+
+constexpr int kMaxDevices = 64;
+int g_dev_state[kMaxDevices];  // 0 unknown, 1 supported, 2 unsupported
+int g_dev_sms[kMaxDevices];
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t fwd_groups(int64_t V) { return ceil_div(ceil_div(V, kBN), kFwdGroup); }
+
+// Vocab columns per backward chunk (a multiple of kBN, at most kVChunk).
+int64_t vchunk(int64_t V) { return std::min<int64_t>(kVChunk, ceil_div(V, kBN) * kBN); }
+
+struct Layout {
+  size_t pm, ps, pb, yt, fwd_end;
+  size_t dx, dh, bwd_end;
+};
+
+Layout layout(int64_t T, int64_t H, int64_t V) {
+  Layout L;
+  const size_t G = static_cast<size_t>(fwd_groups(V));
+  const size_t t = static_cast<size_t>(T);
+  L.pm = kHeader;
+  L.ps = L.pm + align256(G * t * 4);
+  L.pb = L.ps + align256(G * t * 4);
+  L.yt = L.pb + align256(G * t * 4);
+  L.fwd_end = L.yt + align256(t * 4);
+  L.dx = kHeader;
+  L.dh = L.dx + align256(t * static_cast<size_t>(vchunk(V)) * 2);
+  L.bwd_end = L.dh + align256(t * static_cast<size_t>(H) * 4);
+  return L;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+rlk_status check_sizes(int64_t T, int64_t H, int64_t V, float temperature) {
+  if (T < 0 || H <= 0 || V <= 0) return RLK_ERR_INVALID_ARG;
+  if (!std::isfinite(temperature) || !(temperature > 0.f)) return RLK_ERR_INVALID_ARG;
+  if (!std::isfinite(kLog2e / temperature)) return RLK_ERR_INVALID_ARG;
+  if (H % 64 != 0 || H > (int64_t{1} << 20)) return RLK_ERR_UNSUPPORTED_SHAPE;
+  if (V >= (int64_t{1} << 31) || T >= (int64_t{1} << 31)) return RLK_ERR_UNSUPPORTED_SHAPE;
+  return RLK_OK;
+}
+
+// Current device must be compute capability 10.0 (B200, sm_100a code).
+rlk_status check_device(int* num_sms) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) {
+    cudaGetLastError();
+    return RLK_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return RLK_ERR_UNSUPPORTED_DEVICE;
+  if (g_dev_state[dev] == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return RLK_ERR_CUDA;
+    }
+    g_dev_sms[dev] = sms;
+    g_dev_state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  if (g_dev_state[dev] != 1) return RLK_ERR_UNSUPPORTED_DEVICE;
+  *num_sms = g_dev_sms[dev];
+  return RLK_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major matrix with `inner` contiguous
+// elements per row, `outer` rows and a row pitch of `pitch_elems`; boxes of
+// box_inner x box_outer, 128-byte swizzle, zero fill outside the matrix.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K-major operand [rows, K] (K contiguous): one 64 x box_rows box per stage.
+bool map_kmajor(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t pitch,
+                uint32_t box_rows) {
+  return make_map(m, base, K, rows, pitch, 64, box_rows);
+}
+
+// MN-major operand stored [K, MN] (MN contiguous): 64 x 64 boxes.
+bool map_mnmajor(CUtensorMap* m, const void* base, int64_t MN, int64_t K, int64_t pitch) {
+  return make_map(m, base, MN, K, pitch, 64, 64);
+}
+
+Sched make_sched(int64_t M, int64_t N, int64_t K, int group) {
+  Sched s;
+  s.num_m_tiles = static_cast<int>(ceil_div(M, kBM));
+  s.num_n_tiles = static_cast<int>(ceil_div(N, kBN));
+  s.group = group;
+  s.num_groups = static_cast<int>(ceil_div(s.num_n_tiles, group));
+  s.num_units = s.num_m_tiles * s.num_groups;
+  s.num_k_blocks = static_cast<int>(ceil_div(K, kBK));
+  s.a_m_off = s.a_k_off = s.b_n_off = s.b_k_off = 0;
+  s.a_mn_extent = static_cast<int>(M);
+  s.b_mn_extent = static_cast<int>(N);
+  return s;
+}
+
+template <class Epi, bool A_MN, bool B_MN>
+rlk_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const Sched& sc,
+                       const typename Epi::Params& ep, uint32_t* err, cudaStream_t st,
+                       int num_sms) {
+  if (sc.num_units <= 0) return RLK_OK;
+  auto kern = gemm_kernel<Epi, A_MN, B_MN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemBytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  const int grid = std::min(sc.num_units, num_sms);
+  kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, sc, ep, err);
+  return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace rlk
+
+using namespace rlk;
+
+extern "C" {
+
+size_t rlk_linear_logp_workspace_bytes(int64_t T, int64_t H, int64_t V, int for_backward) {
+  if (check_sizes(T, H, V, 1.0f) != RLK_OK) return 0;
+  const Layout L = layout(T, H, V);
+  return for_backward ? std::max(L.fwd_end, L.bwd_end) : L.fwd_end;
+}
+
+rlk_status rlk_linear_logp_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                               int64_t T, int64_t H, int64_t V, float temperature, float* logp,
+                               float* entropy, float* lse, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (T == 0) return RLK_OK;
+  if (!hidden || !W || !targets || !logp || !entropy || !lse || !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(workspace, 256) ||
+      !aligned(targets, 8) || !aligned(logp, 4) || !aligned(entropy, 4) || !aligned(lse, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);
+  if (workspace_bytes < L.fwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  CUtensorMap mh, mw;
+  if (!map_kmajor(&mh, hidden, H, T, H, kBM) || !map_kmajor(&mw, W, H, V, H, kBN))
+    return RLK_ERR_CUDA;
+
+  Sched sc = make_sched(T, V, H, kFwdGroup);
+  EpiFwd::Params ep;
+  ep.targets = targets;
+  ep.part_m = reinterpret_cast<float*>(ws + L.pm);
+  ep.part_s = reinterpret_cast<float*>(ws + L.ps);
+  ep.part_b = reinterpret_cast<float*>(ws + L.pb);
+  ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
+  ep.T = static_cast<int>(T);
+  ep.V = static_cast<int>(V);
+  ep.scale_log2 = kLog2e / temperature;
+  if ((s = launch_gemm<EpiFwd, false, false>(mh, mw, sc, ep, err, st, sms)) != RLK_OK) return s;
+
+  const int G = sc.num_groups;
+  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, st>>>(
+      ep.part_m, ep.part_s, ep.part_b, ep.ytgt, targets, static_cast<int>(T),
+      static_cast<int>(V), G, logp, entropy, lse, err);
+  if (cudaGetLastError() != cudaSuccess) return RLK_ERR_CUDA;
+  g_calls[0].fetch_add(1);
+  return RLK_OK;
+}
+
+rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                               int64_t T, int64_t H, int64_t V, float temperature,
+                               const float* lse, const float* entropy, const float* dlogp,
+                               const float* dentropy, rlk_bf16* dHidden, float* dW,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (!dW) return RLK_ERR_INVALID_ARG;
+  if (!aligned(dW, 16)) return RLK_ERR_MISALIGNED;
+  int sms = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if ((s = check_device(&sms)) != RLK_OK) return s;
+    if (cudaMemsetAsync(dW, 0, static_cast<size_t>(V) * H * 4, st) != cudaSuccess)
+      return RLK_ERR_CUDA;
+    g_calls[1].fetch_add(1);
+    return RLK_OK;
+  }
+  if (!hidden || !W || !targets || !lse || !entropy || !dlogp || !dentropy || !dHidden ||
+      !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(dHidden, 16) ||
+      !aligned(workspace, 256) || !aligned(targets, 8) || !aligned(lse, 4) ||
+      !aligned(entropy, 4) || !aligned(dlogp, 4) || !aligned(dentropy, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);
+  if (workspace_bytes < L.bwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  __nv_bfloat16* dX = reinterpret_cast<__nv_bfloat16*>(ws + L.dx);
+  float* dh_acc = reinterpret_cast<float*>(ws + L.dh);
+  const int64_t ldx = vchunk(V);
+  const int64_t nchunks = ceil_div(V, ldx);
+
+  CUtensorMap m_hid_k, m_w_k, m_w_mn, m_hid_mn;
+  if (!map_kmajor(&m_hid_k, hidden, H, T, H, kBM) || !map_kmajor(&m_w_k, W, H, V, H, kBN) ||
+      !map_mnmajor(&m_w_mn, W, H, V, H) || !map_mnmajor(&m_hid_mn, hidden, H, T, H))
+    return RLK_ERR_CUDA;
+
+  for (int64_t c = 0; c < nchunks; ++c) {
+    const int64_t c0 = c * ldx;
+    const int64_t valid = std::min(ldx, V - c0);
+
+    // (1) recompute the chunk's logits and write its bf16 dlogits to dX.
+    Sched s1 = make_sched(T, valid, H, 1);
+    s1.b_n_off = static_cast<int>(c0);
+    s1.b_mn_extent = static_cast<int>(V);
+    EpiDlogits::Params p1;
+    p1.targets = targets;
+    p1.lse = lse;
+    p1.entropy = entropy;
+    p1.dlogp = dlogp;
+    p1.dentropy = dentropy;
+    p1.dX = dX;
+    p1.err = err;
+    p1.T = static_cast<int>(T);
+    p1.V = static_cast<int>(V);
+    p1.c0 = static_cast<int>(c0);
+    p1.ldx = static_cast<int>(ldx);
+    p1.scale_log2 = kLog2e / temperature;
+    p1.inv_tau = 1.0f / temperature;
+    if ((s = launch_gemm<EpiDlogits, false, false>(m_hid_k, m_w_k, s1, p1, err, st, sms)) !=
+        RLK_OK)
+      return s;
+
+    CUtensorMap m_dx_k, m_dx_mn;
+    if (!map_kmajor(&m_dx_k, dX, valid, T, ldx, kBM) || !map_mnmajor(&m_dx_mn, dX, valid, T, ldx))
+      return RLK_ERR_CUDA;
+
+    // (2) dHidden += dX[T, valid] . W[c0 : c0 + valid, :]
+    Sched s2 = make_sched(T, H, valid, 1);
+    s2.b_k_off = static_cast<int>(c0);
+    EpiDh::Params p2;
+    p2.acc = dh_acc;
+    p2.out = reinterpret_cast<__nv_bfloat16*>(dHidden);
+    p2.T = static_cast<int>(T);
+    p2.H = static_cast<int>(H);
+    p2.mode = nchunks == 1 ? EpiDh::kOnly
+              : c == 0     ? EpiDh::kFirst
+              : c == nchunks - 1 ? EpiDh::kLast
+                                 : EpiDh::kMiddle;
+    if ((s = launch_gemm<EpiDh, false, true>(m_dx_k, m_w_mn, s2, p2, err, st, sms)) != RLK_OK)
+      return s;
+
+    // (3) dW[c0 : c0 + valid, :] = dX[T, valid]^T . hidden[T, H]
+    Sched s3 = make_sched(valid, H, T, 1);
+    EpiStore::Params p3;
+    p3.out = dW + static_cast<size_t>(c0) * H;
+    p3.rows = static_cast<int>(valid);
+    p3.ncols = static_cast<int>(H);
+    p3.ld = static_cast<int>(H);
+    if ((s = launch_gemm<EpiStore, true, true>(m_dx_mn, m_hid_mn, s3, p3, err, st, sms)) !=
+        RLK_OK)
+      return s;
+  }
+  g_calls[1].fetch_add(1);
+  return RLK_OK;
+}
+
+size_t rlk_gemm_workspace_bytes(void) { return kHeader; }
+
+rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, int64_t N,
+                             int64_t K, int a_mn_major, int b_mn_major, float* C,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return RLK_ERR_INVALID_ARG;
+  if (M % 8 || N % 8 || K % 8 || M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) ||
+      K >= (int64_t{1} << 31))
+    return RLK_ERR_UNSUPPORTED_SHAPE;
+  if (!A || !B || !C || !workspace) return RLK_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(workspace, 256))
+    return RLK_ERR_MISALIGNED;
+  if (workspace_bytes < kHeader) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  rlk_status s = check_device(&sms);
+  if (s != RLK_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(workspace);
+
+  CUtensorMap ma, mb;
+  bool ok = a_mn_major ? map_mnmajor(&ma, A, M, K, M) : map_kmajor(&ma, A, K, M, K, kBM);
+  ok = ok && (b_mn_major ? map_mnmajor(&mb, B, N, K, N) : map_kmajor(&mb, B, K, N, K, kBN));
+  if (!ok) return RLK_ERR_CUDA;
+  Sched sc = make_sched(M, N, K, 1);
+  EpiStore::Params ep;
+  ep.out = C;
+  ep.rows = static_cast<int>(M);
+  ep.ncols = static_cast<int>(N);
+  ep.ld = static_cast<int>(N);
+  if (!a_mn_major && !b_mn_major)
+    s = launch_gemm<EpiStore, false, false>(ma, mb, sc, ep, err, st, sms);
+  else if (!a_mn_major && b_mn_major)
+    s = launch_gemm<EpiStore, false, true>(ma, mb, sc, ep, err, st, sms);
+  else if (a_mn_major && !b_mn_major)
+    s = launch_gemm<EpiStore, true, false>(ma, mb, sc, ep, err, st, sms);
+  else
+    s = launch_gemm<EpiStore, true, true>(ma, mb, sc, ep, err, st, sms);
+  if (s == RLK_OK) g_calls[2].fetch_add(1);
+  return s;
+}
+
+const char* rlk_backend_id(void) { return "rlk.linear_logp.bitwise.sm100a.v1"; }
+
+uint64_t rlk_call_count(int which) {
+  if (which < 0 || which > 2) return 0;
+  return g_calls[which].load();
+}
+
+rlk_status rlk_read_device_error(void* workspace, uint32_t* flags, void* stream) {
+  if (!workspace || !flags) return RLK_ERR_INVALID_ARG;
+  if (!aligned(workspace, 4)) return RLK_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  *flags = v;
+  return RLK_OK;
+}
+
+const char* rlk_status_string(rlk_status status) {
+  switch (status) {
+    case RLK_OK: return "RLK_OK";
+    case RLK_ERR_INVALID_ARG: return "RLK_ERR_INVALID_ARG";
+    case RLK_ERR_UNSUPPORTED_SHAPE: return "RLK_ERR_UNSUPPORTED_SHAPE";
+    case RLK_ERR_MISALIGNED: return "RLK_ERR_MISALIGNED";
+    case RLK_ERR_WORKSPACE_TOO_SMALL: return "RLK_ERR_WORKSPACE_TOO_SMALL";
+    case RLK_ERR_UNSUPPORTED_DEVICE: return "RLK_ERR_UNSUPPORTED_DEVICE";
+    case RLK_ERR_CUDA: return "RLK_ERR_CUDA";
+  }
+  return "RLK_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,613 @@
+// rlk_gemm.cuh -- the one tensor-core mainloop behind every linear-logp
+// kernel, and the epilogues that turn its accumulator tiles into the
+// operator's results.
+//
+// Mainloop.  D[M,N] = sum_k A[m,k] B[n,k] in 128 x 256 output tiles, bf16
+// operands, fp32 accumulation in tensor memory (TMEM).  Persistent CTAs (one
+// per SM, 192 threads, ~193 KB of shared memory) walk a static list of
+// "units"; a unit is one 128-row M tile and `group` consecutive 256-column N
+// tiles, processed in ascending order.  Warp roles:
+//   warp 0     TMA producer: 4-stage ring of (A 128x64, B 256x64) bf16 tiles,
+//              128-byte swizzled, one mbarrier pair per stage;
+//   warp 1     allocates 512 TMEM columns (two 256-column fp32 accumulators)
+//              and issues tcgen05.mma (M=128, N=256, K=16) from one thread;
+//   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane),
+//              reads it 32 columns at a time with tcgen05.ld and hands the
+//              values to the epilogue policy.
+// The accumulator is double buffered so the epilogue of tile i overlaps the
+// MMAs of tile i+1.  Every pipeline wait is bounded (rlk_ptx.cuh).
+//
+// Operands may be K-major (row of A / B contiguous along K) or MN-major
+// (contiguous along M / N); the instruction descriptor's transpose bits and
+// the shared-memory descriptors handle both, so the backward GEMMs read
+// dlogits, W and hidden in place without transposed copies.
+//
+// Batch invariance.  Each output element is produced by one CTA with a K
+// loop of fixed order and fixed instruction shape, and every epilogue works
+// row by row; nothing depends on how many rows the problem has or on which
+// CTA runs a unit.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "rlk_ptx.cuh"
+
+namespace rlk {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kAStage = kBM * kBK * 2;  // 16 KB
+constexpr uint32_t kBStage = kBN * kBK * 2;  // 32 KB
+constexpr uint32_t kBox = 64 * 64 * 2;       // one MN-major 64x64 box, 8 KB
+constexpr int kNumBars = 2 * kStages + 5;
+constexpr size_t kSmemBytes = 1024 + kStages * (kAStage + kBStage) + kNumBars * 8 + 16;
+
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
+constexpr float kLn2 = 0.6931471805599453f;    // ln(2)
+constexpr float kMaskLogit = -1.0e30f;         // stands for -inf without producing NaN
+
+struct Sched {
+  int num_m_tiles;   // ceil(M / kBM)
+  int num_n_tiles;   // ceil(N / kBN)
+  int group;         // N tiles per unit
+  int num_groups;    // ceil(num_n_tiles / group)
+  int num_units;     // num_m_tiles * num_groups
+  int num_k_blocks;  // ceil(K / kBK)
+  int a_m_off, a_k_off;  // tensor-map coordinate offsets of A
+  int b_n_off, b_k_off;  // and of B
+  int a_mn_extent;   // extent of A's M coordinate in its tensor map
+  int b_mn_extent;   // extent of B's N coordinate in its tensor map
+};
+
+__device__ __forceinline__ void decode_unit(const Sched& sc, int u, int& mt, int& g, int& nt0,
+                                            int& nt1) {
+  mt = u % sc.num_m_tiles;
+  g = u / sc.num_m_tiles;
+  nt0 = g * sc.group;
+  nt1 = min(nt0 + sc.group, sc.num_n_tiles);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// =====================================================================
+// Epilogue policies.  Each provides Params, State and
+//   begin_unit(p, st, row, mt, g)   once per unit, row = global M index
+//   tile(p, st, taddr, nt)          once per 128x256 accumulator tile
+//   end_unit(p, st, g)              once per unit
+// =====================================================================
+
+// Forward: per row, over the unit's vocab tiles in ascending order, keep the
+// online triple in base-2 units of y = x * log2(e) / tau:
+//   m = max y,  s = sum 2^(y - m),  b = sum 2^(y - m) (y - m)
+// and pick up y at the row's target column.  The triple of each (row,
+// vocab split) goes to the workspace for the fixed-order combine.
+struct EpiFwd {
+  struct Params {
+    const int64_t* targets;
+    float* part_m;
+    float* part_s;
+    float* part_b;
+    float* ytgt;
+    int T;
+    int V;
+    float scale_log2;  // log2(e) / tau
+  };
+  struct State {
+    float m, s, b;
+    int64_t tgt;
+    int row;
+    bool valid;
+  };
+
+  __device__ static void begin_unit(const Params& p, State& st, int row, int, int) {
+    st.row = row;
+    st.valid = row < p.T;
+    st.tgt = st.valid ? p.targets[row] : -1;
+    st.m = kMaskLogit;
+    st.s = 0.f;
+    st.b = 0.f;
+  }
+
+  __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      const int col0 = nt * kBN + c * 32;
+      float y[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(r[j]) * p.scale_log2;
+      if (col0 + 32 > p.V) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j >= p.V) y[j] = kMaskLogit;
+      }
+      const int64_t d = st.tgt - col0;
+      if (d >= 0 && d < 32) {
+        float yt = y[0];
+#pragma unroll
+        for (int j = 1; j < 32; ++j) yt = (j == d) ? y[j] : yt;
+        p.ytgt[st.row] = yt;
+      }
+      float cm = y[0];
+#pragma unroll
+      for (int j = 1; j < 32; ++j) cm = fmaxf(cm, y[j]);
+      const float mn = fmaxf(st.m, cm);
+      const float a = ex2_approx(st.m - mn);
+      st.b = a * fmaf(st.m - mn, st.s, st.b);
+      st.s = st.s * a;
+      st.m = mn;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float dd = y[j] - mn;
+        const float e = ex2_approx(dd);
+        st.s += e;
+        st.b = fmaf(e, dd, st.b);
+      }
+    }
+  }
+
+  __device__ static void end_unit(const Params& p, State& st, int g) {
+    if (st.valid) {
+      const size_t i = static_cast<size_t>(g) * p.T + st.row;
+      p.part_m[i] = st.m;
+      p.part_s[i] = st.s;
+      p.part_b[i] = st.b;
+    }
+  }
+};
+
+// Backward recompute: the same logits tile, turned into bf16 dlogits
+//   dx = (dlogp (1[v = target] - p) - dentropy p (z - E_p z)) / tau
+// with p = 2^(y - lse log2 e), written to the chunk buffer dX[T, ldx]
+// (columns are local to the vocab chunk starting at c0).
+struct EpiDlogits {
+  struct Params {
+    const int64_t* targets;
+    const float* lse;
+    const float* entropy;
+    const float* dlogp;
+    const float* dentropy;
+    __nv_bfloat16* dX;
+    uint32_t* err;
+    int T;
+    int V;
+    int c0;
+    int ldx;
+    float scale_log2;  // log2(e) / tau
+    float inv_tau;
+  };
+  struct State {
+    float A, k1, k2, hot;
+    int64_t tloc;
+    int row;
+    bool valid;
+  };
+
+  __device__ static void begin_unit(const Params& p, State& st, int row, int, int) {
+    st.row = row;
+    st.valid = row < p.T;
+    st.A = 0.f;
+    st.k1 = st.k2 = st.hot = 0.f;
+    st.tloc = -1;
+    if (st.valid) {
+      const float lse = p.lse[row], ent = p.entropy[row];
+      const float dl = p.dlogp[row], de = p.dentropy[row];
+      const int64_t tg = p.targets[row];
+      const float ez = lse - ent;  // E_p z
+      st.A = lse * kLog2e;
+      // dx = hot*1[v=target] - p*(k1 + k2*y)
+      st.k1 = p.inv_tau * (dl - de * ez);
+      st.k2 = p.inv_tau * de * kLn2;
+      st.hot = p.inv_tau * dl;
+      if (tg >= 0 && tg < p.V) {
+        st.tloc = tg - p.c0;
+      } else if (p.c0 == 0) {
+        atomicOr(p.err, kDevErrTarget);
+      }
+    }
+  }
+
+  __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      const int loc0 = nt * kBN + c * 32;
+      const int col0 = p.c0 + loc0;
+      float dx[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float y = __uint_as_float(r[j]) * p.scale_log2;
+        const float pr = ex2_approx(y - st.A);
+        dx[j] = -pr * fmaf(st.k2, y, st.k1);
+      }
+      if (col0 + 32 > p.V) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j >= p.V) dx[j] = 0.f;
+      }
+      const int64_t d = st.tloc - loc0;
+      if (d >= 0 && d < 32) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dx[j] = (j == d) ? dx[j] + st.hot : dx[j];
+      }
+      if (st.valid) {
+        uint4* dst = reinterpret_cast<uint4*>(p.dX + static_cast<size_t>(st.row) * p.ldx + loc0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(dx[8 * q + 0], dx[8 * q + 1]);
+          w.y = pack_bf16x2(dx[8 * q + 2], dx[8 * q + 3]);
+          w.z = pack_bf16x2(dx[8 * q + 4], dx[8 * q + 5]);
+          w.w = pack_bf16x2(dx[8 * q + 6], dx[8 * q + 7]);
+          dst[q] = w;
+        }
+      }
+    }
+  }
+
+  __device__ static void end_unit(const Params&, State&, int) {}
+};
+
+// dHidden: acc[T,H] (fp32 workspace) collects the vocab chunks in ascending
+// order: chunk 0 stores, later chunks add (old + new), the last chunk writes
+// the bf16 result.
+struct EpiDh {
+  enum Mode { kFirst = 0, kMiddle = 1, kLast = 2, kOnly = 3 };
+  struct Params {
+    float* acc;
+    __nv_bfloat16* out;
+    int T;
+    int H;
+    int mode;
+  };
+  struct State {
+    int row;
+    bool valid;
+  };
+
+  __device__ static void begin_unit(const Params& p, State& st, int row, int, int) {
+    st.row = row;
+    st.valid = row < p.T;
+  }
+
+  __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      const int col0 = nt * kBN + c * 32;
+      if (col0 >= p.H) break;  // warp-uniform
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      if (!st.valid) continue;
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      const size_t off = static_cast<size_t>(st.row) * p.H + col0;
+      float4* pa = reinterpret_cast<float4*>(p.acc + off);
+      if (p.mode == kMiddle || p.mode == kLast) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 o = pa[q];
+          v[4 * q + 0] = o.x + v[4 * q + 0];
+          v[4 * q + 1] = o.y + v[4 * q + 1];
+          v[4 * q + 2] = o.z + v[4 * q + 2];
+          v[4 * q + 3] = o.w + v[4 * q + 3];
+        }
+      }
+      if (p.mode == kFirst || p.mode == kMiddle) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          pa[q] = make_float4(v[4 * q + 0], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+          w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+          w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+          w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+          dst[q] = w;
+        }
+      }
+    }
+  }
+
+  __device__ static void end_unit(const Params&, State&, int) {}
+};
+
+// Plain fp32 store of the tile into out[rows, ld] (dW rows of one vocab
+// chunk, or the self-check GEMM's C).  Columns >= ncols are skipped.
+struct EpiStore {
+  struct Params {
+    float* out;
+    int rows;
+    int ncols;
+    int ld;
+  };
+  struct State {
+    int row;
+    bool valid;
+  };
+
+  __device__ static void begin_unit(const Params& p, State& st, int row, int, int) {
+    st.row = row;
+    st.valid = row < p.rows;
+  }
+
+  __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt) {
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      const int col0 = nt * kBN + c * 32;
+      if (col0 >= p.ncols) break;  // warp-uniform
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      if (!st.valid) continue;
+      float* dst = p.out + static_cast<size_t>(st.row) * p.ld + col0;
+      if (col0 + 32 <= p.ncols) {
+        float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          d4[q] = make_float4(__uint_as_float(r[4 * q + 0]), __uint_as_float(r[4 * q + 1]),
+                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < p.ncols) dst[j] = __uint_as_float(r[j]);
+      }
+    }
+  }
+
+  __device__ static void end_unit(const Params&, State&, int) {}
+};
+
+// =====================================================================
+// The persistent kernel.
+// =====================================================================
+template <class Epi, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Sched sc, const typename Epi::Params ep, uint32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + kStages * kAStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * (kAStage + kBStage));
+  const uint32_t bar0 = smem_u32(bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  uint32_t issued = 0;  // producer: k-blocks whose loads were issued
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < sc.num_units; u += gridDim.x) {
+        int mt, g, nt0, nt1;
+        decode_unit(sc, u, mt, g, nt0, nt1);
+        for (int nt = nt0; ok && nt < nt1; ++nt) {
+          for (int kb = 0; kb < sc.num_k_blocks; ++kb) {
+            const int s = issued % kStages;
+            const uint32_t ph = (issued / kStages) & 1u;
+            if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dA = sA + s * kAStage;
+            const uint32_t dB = sB + s * kBStage;
+            const int ka = sc.a_k_off + kb * kBK;
+            const int kbb = sc.b_k_off + kb * kBK;
+            const int m0 = sc.a_m_off + mt * kBM;
+            const int n0 = sc.b_n_off + nt * kBN;
+            uint32_t bytes = 0;
+            if (!A_MN) {
+              bytes += kAStage;
+            } else {
+#pragma unroll
+              for (int j = 0; j < kBM / 64; ++j)
+                if (m0 + 64 * j < sc.a_mn_extent) bytes += kBox;
+            }
+            if (!B_MN) {
+              bytes += kBStage;
+            } else {
+#pragma unroll
+              for (int j = 0; j < kBN / 64; ++j)
+                if (n0 + 64 * j < sc.b_mn_extent) bytes += kBox;
+            }
+            mbar_arrive_expect_tx(full_bar(s), bytes);
+            if (!A_MN) {
+              tma_load_2d(dA, &tmA, full_bar(s), ka, m0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < kBM / 64; ++j)
+                if (m0 + 64 * j < sc.a_mn_extent)
+                  tma_load_2d(dA + j * kBox, &tmA, full_bar(s), m0 + 64 * j, ka);
+            }
+            if (!B_MN) {
+              tma_load_2d(dB, &tmB, full_bar(s), kbb, n0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < kBN / 64; ++j)
+                if (n0 + 64 * j < sc.b_mn_extent)
+                  tma_load_2d(dB + j * kBox, &tmB, full_bar(s), n0 + 64 * j, kbb);
+            }
+            ++issued;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, A_MN, B_MN);
+      constexpr uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
+      constexpr uint32_t a_kstep = A_MN ? 2048u : 32u, b_kstep = B_MN ? 2048u : 32u;
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < sc.num_units; u += gridDim.x) {
+        int mt, g, nt0, nt1;
+        decode_unit(sc, u, mt, g, nt0, nt1);
+        for (int nt = nt0; ok && nt < nt1; ++nt, ++tc) {
+          const int acc = tc & 1;
+          const uint32_t use = tc >> 1;
+          if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * kBN;
+          for (int kb = 0; kb < sc.num_k_blocks; ++kb, ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1u;
+            if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = sA + s * kAStage, b0 = sB + s * kBStage;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(a0 + k * a_kstep, a_lbo, 1024u);
+              const uint64_t bd = smem_desc_sw128(b0 + k * b_kstep, b_lbo, 1024u);
+              umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
+            umma_commit(empty_bar(s));
+          }
+          if (ok) umma_commit(tfull_bar(acc));
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    uint32_t tc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < sc.num_units; u += gridDim.x) {
+      int mt, g, nt0, nt1;
+      decode_unit(sc, u, mt, g, nt0, nt1);
+      typename Epi::State st;
+      Epi::begin_unit(ep, st, mt * kBM + row_in_tile, mt, g);
+      for (int nt = nt0; nt < nt1; ++nt, ++tc) {
+        const int acc = tc & 1;
+        const uint32_t use = tc >> 1;
+        int w = 1;
+        if (lane == 0) w = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, err) ? 1 : 0;
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN;
+        Epi::tile(ep, st, taddr, nt);
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+      }
+      if (ok) Epi::end_unit(ep, st, g);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // Unwind after a timed-out wait: let every TMA load still in flight land
+    // and every issued MMA finish before the memory they touch goes away.
+    if (warp == 0 && lane == 0) {
+      const uint32_t first = issued > static_cast<uint32_t>(kStages) ? issued - kStages : 0u;
+      for (uint32_t i = first; i < issued; ++i)
+        mbar_wait_drain(full_bar(i % kStages), (i / kStages) & 1u);
+    }
+    if (warp == 1 && lane == 0) {
+      umma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+    __syncthreads();
+  }
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// Fixed-order merge of the forward's per-split triples, one thread per row:
+// lse = ln2 (M + log2 S), entropy = ln2 (log2 S - B / S),
+// logp = ln2 (y_target - M - log2 S).
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ pm,
+                                                      const float* __restrict__ ps,
+                                                      const float* __restrict__ pb,
+                                                      const float* __restrict__ ytgt,
+                                                      const int64_t* __restrict__ targets, int T,
+                                                      int V, int G, float* __restrict__ logp,
+                                                      float* __restrict__ entropy,
+                                                      float* __restrict__ lse, uint32_t* err) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  float M = kMaskLogit, S = 0.f, B = 0.f;
+  for (int g = 0; g < G; ++g) {
+    const size_t i = static_cast<size_t>(g) * T + t;
+    const float m = pm[i], s = ps[i], b = pb[i];
+    const float mn = fmaxf(M, m);
+    const float a1 = ex2_approx(M - mn);
+    const float a2 = ex2_approx(m - mn);
+    B = a1 * fmaf(M - mn, S, B) + a2 * fmaf(m - mn, s, b);
+    S = a1 * S + a2 * s;
+    M = mn;
+  }
+  const float l2s = log2f(S);
+  lse[t] = kLn2 * (M + l2s);
+  entropy[t] = kLn2 * (l2s - B / S);
+  const int64_t tg = targets[t];
+  if (tg < 0 || tg >= V) {
+    logp[t] = __int_as_float(0x7fc00000);
+    atomicOr(err, kDevErrTarget);
+  } else {
+    logp[t] = kLn2 * ((ytgt[t] - M) - l2s);
+  }
+}
+
+}  // namespace rlk

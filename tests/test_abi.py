@@ -1,0 +1,121 @@
+"""C-ABI checks that need no GPU: the library builds, loads and exports every
+function include/rlk.h declares; argument validation returns the documented
+status before any CUDA work; provenance strings."""
+import ctypes
+
+import pytest
+import torch
+
+from invariant_lm_head_gemm_b200 import binding, build
+
+OK, INVALID, SHAPE, MISALIGNED, WS_SMALL, DEVICE, CUDA = range(7)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return binding.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = binding.declared_functions()
+    assert {"rlk_linear_logp_fwd", "rlk_linear_logp_bwd",
+            "rlk_linear_logp_workspace_bytes"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_backend_id(L):
+    assert [binding.status_string(s) for s in range(7)] == [
+        "RLK_OK", "RLK_ERR_INVALID_ARG", "RLK_ERR_UNSUPPORTED_SHAPE", "RLK_ERR_MISALIGNED",
+        "RLK_ERR_WORKSPACE_TOO_SMALL", "RLK_ERR_UNSUPPORTED_DEVICE", "RLK_ERR_CUDA"]
+    assert binding.status_string(99) == "RLK_ERR_UNKNOWN"
+    assert binding.backend_id() == "rlk.linear_logp.bitwise.sm100a.v1"
+    assert binding.call_count(7) == 0
+
+
+def test_workspace_bytes(L):
+    T, H, V = 5200, 4096, 151936
+    fwd = binding.workspace_bytes(T, H, V, False)
+    both = binding.workspace_bytes(T, H, V, True)
+    # fwd: 256-byte header + 3 x [297 splits x T] fp32 partials + [T] target logits
+    def a(x):
+        return (x + 255) // 256 * 256
+    assert fwd == 256 + 3 * a(297 * T * 4) + a(T * 4)
+    # bwd: header + [T, 8192] bf16 dlogits chunk + [T, H] fp32 dHidden accumulator
+    assert both == max(fwd, 256 + a(T * 8192 * 2) + a(T * H * 4))
+    assert binding.workspace_bytes(4, 100, 10) == 0          # H % 64 != 0
+    assert binding.workspace_bytes(4, 64, 0) == 0
+    assert binding.workspace_bytes(0, 64, 10) > 0
+    # small V: the chunk buffer shrinks to V rounded up to 256 columns
+    assert binding.workspace_bytes(8, 64, 300, True) >= 256 + 8 * 512 * 2 + 8 * 64 * 4
+
+
+A16 = 0x10000        # fake, never dereferenced: validation must fail first
+A256 = 0x20000
+
+
+def _fwd(L, hidden=A16, W=A16, targets=A16, T=4, H=64, V=10, tau=1.0, logp=A16, ent=A16,
+         lse=A16, ws=A256, wsb=1 << 30):
+    return L.rlk_linear_logp_fwd(hidden, W, targets, T, H, V, tau, logp, ent, lse, ws, wsb, None)
+
+
+def _bwd(L, dW=A16, dH=A16, T=4, H=64, V=10, tau=1.0, ws=A256, wsb=1 << 30, hidden=A16):
+    return L.rlk_linear_logp_bwd(hidden, A16, A16, T, H, V, tau, A16, A16, A16, A16, dH, dW,
+                                 ws, wsb, None)
+
+
+def test_forward_argument_errors(L):
+    assert _fwd(L, T=-1) == INVALID
+    assert _fwd(L, H=0) == INVALID
+    assert _fwd(L, V=0) == INVALID
+    for tau in (0.0, -1.0, float("nan"), float("inf"), 1e-45):
+        assert _fwd(L, tau=tau) == INVALID, tau
+    assert _fwd(L, H=100) == SHAPE
+    assert _fwd(L, H=64 * (1 << 15)) == SHAPE
+    assert _fwd(L, V=1 << 31) == SHAPE
+    assert _fwd(L, T=0, hidden=None, W=None, targets=None) == OK     # empty batch: no-op
+    for k in ("hidden", "W", "targets", "logp", "ent", "lse", "ws"):
+        assert _fwd(L, **{k: None}) == INVALID, k
+    assert _fwd(L, hidden=A16 + 8) == MISALIGNED
+    assert _fwd(L, W=A16 + 2) == MISALIGNED
+    assert _fwd(L, ws=A256 + 16) == MISALIGNED
+    assert _fwd(L, targets=A16 + 4) == MISALIGNED
+    assert _fwd(L, logp=A16 + 2) == MISALIGNED
+    need = binding.workspace_bytes(4, 64, 10, False)
+    assert _fwd(L, wsb=need - 1) == WS_SMALL
+
+
+def test_backward_argument_errors(L):
+    assert _bwd(L, T=-2) == INVALID
+    assert _bwd(L, tau=0.0) == INVALID
+    assert _bwd(L, H=96) == SHAPE
+    assert _bwd(L, dW=None) == INVALID
+    assert _bwd(L, dW=A16 + 4) == MISALIGNED
+    assert _bwd(L, dH=None) == INVALID
+    assert _bwd(L, hidden=None) == INVALID
+    assert _bwd(L, dH=A16 + 2) == MISALIGNED
+    need = binding.workspace_bytes(4, 64, 10, True)
+    assert _bwd(L, wsb=need - 1) == WS_SMALL
+
+
+def test_gemm_argument_errors(L):
+    g = L.rlk_gemm_bf16_f32
+    assert g(A16, A16, 0, 8, 8, 0, 0, A16, A256, 256, None) == INVALID
+    assert g(A16, A16, 12, 8, 8, 0, 0, A16, A256, 256, None) == SHAPE
+    assert g(None, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == INVALID
+    assert g(A16 + 2, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == MISALIGNED
+    assert g(A16, A16, 8, 8, 8, 0, 0, A16, A256, 255, None) == WS_SMALL
+    v = ctypes.c_uint32(0)
+    assert L.rlk_read_device_error(None, ctypes.byref(v), None) == INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU refusal")
+def test_valid_call_without_a_gpu_is_refused(L):
+    # every argument is valid, so the only thing left to fail is the device:
+    # the library must refuse (fail closed), not fall back to anything
+    assert _fwd(L) == DEVICE
+    assert _bwd(L) == DEVICE
+    assert _bwd(L, T=0) == DEVICE
+    assert L.rlk_gemm_bf16_f32(A16, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == DEVICE
+    assert binding.call_count(0) == 0 and binding.call_count(1) == 0

@@ -1,0 +1,50 @@
+"""The tensor-core mainloop on its own (self-check entry rlk_gemm_bf16_f32),
+against a float64 matmul of the same bf16 inputs, for all four operand
+majorness combinations and ragged shapes."""
+import pytest
+import torch
+
+from invariant_lm_head_gemm_b200 import binding
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(128, 256, 64), (8, 8, 8), (200, 264, 136), (136, 520, 4096), (1024, 1024, 1024),
+          (256, 768, 8192)]
+
+
+def _diagnose(C, ref):
+    d = (C - ref).abs()
+    i = int(d.argmax())
+    return ("max|d|=%.3g at %s; C[:3,:3]=%s ref[:3,:3]=%s; rel err vs ref^T-shaped=%s" % (
+        float(d.max()), divmod(i, C.shape[1]), C[:3, :3].tolist(), ref[:3, :3].tolist(),
+        "n/a" if C.shape[0] != C.shape[1] else
+        "%.3g" % float((C - ref.t()).norm() / ref.norm())))
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "M%dN%dK%d" % s)
+@pytest.mark.parametrize("a_mn", [0, 1])
+@pytest.mark.parametrize("b_mn", [0, 1])
+def test_gemm_matches_fp64(shape, a_mn, b_mn):
+    M, N, K = shape
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K + 11 * a_mn + 13 * b_mn)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16)
+    A_st = A.t().contiguous() if a_mn else A
+    B_st = B.t().contiguous() if b_mn else B
+    C, ws = binding.rlk_gemm_bf16_f32(A_st.cuda(), B_st.cuda(), bool(a_mn), bool(b_mn))
+    torch.cuda.synchronize()
+    assert binding.rlk_read_device_error(ws) == 0
+    ref = A.double() @ B.double().t()
+    Cc = C.cpu().double()
+    err = float((Cc - ref).norm() / ref.norm())
+    assert err < 1e-5, _diagnose(Cc, ref)
+
+
+def test_gemm_repeatable():
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(512, 2048, generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(768, 2048, generator=g).to(torch.bfloat16).cuda()
+    C0, _ = binding.rlk_gemm_bf16_f32(A, B)
+    for _ in range(3):
+        C1, _ = binding.rlk_gemm_bf16_f32(A, B)
+        assert torch.equal(C0, C1)
