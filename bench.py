@@ -348,6 +348,37 @@ def run_ours(args):
     return 0
 
 
+def run_profile(args):
+    """A few calls of one pass (fwd or fwd+bwd) on a smaller seeded case, for
+    ncu captures; prints nothing that is a benchmark number."""
+    import torch
+
+    from invariant_lm_head_gemm_b200 import binding
+    from invariant_lm_head_gemm_b200 import workloads as wl
+
+    T, H, V = args.T, 4096, args.V
+    hidden, targets = wl.make_rows(5, T, H, V)
+    W = wl.make_weight(5, V, H)
+    dev = torch.device("cuda", 0)
+
+    def bf(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    hid, Wd = bf(hidden), bf(W)
+    tg = torch.from_numpy(targets).to(dev)
+    dl = torch.ones(T, device=dev)
+    de = torch.full((T,), 1e-3, device=dev)
+    ws = binding.make_workspace(T, H, V, True, dev)
+    for _ in range(args.iters):
+        logp, ent, lse = binding.rlk_linear_logp_fwd(hid, Wd, tg, 1.0, ws)
+        if args.profile == "bwd":
+            binding.rlk_linear_logp_bwd(hid, Wd, tg, 1.0, lse, ent, dl, de, ws)
+    torch.cuda.synchronize()
+    print("profile case done: %s T=%d H=%d V=%d iters=%d flags=%d" % (
+        args.profile, T, H, V, args.iters, binding.rlk_read_device_error(ws)))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -357,7 +388,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=48)
     ap.add_argument("--ref-rows", type=int, default=2)
+    ap.add_argument("--profile", choices=["fwd", "bwd"], default=None,
+                    help="run a small case for an ncu capture instead of the benchmark")
+    ap.add_argument("--T", type=int, default=2048, help="rows of the --profile case")
+    ap.add_argument("--V", type=int, default=32768, help="vocab of the --profile case")
+    ap.add_argument("--iters", type=int, default=3, help="calls in the --profile case")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
