@@ -112,6 +112,30 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
                                const float* dentropy, rlk_bf16* dHidden, float* dW,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* Forward with no workspace argument and no allocation anywhere.  The pages
+ * have no counterpart: this entry exists for callers that cannot allocate
+ * device memory -- code running inside a host framework that owns every
+ * device byte (a serving engine with a pre-reserved memory pool, a plugin
+ * host that forbids allocation calls) or that cannot size a workspace ahead
+ * of time.  Arguments and results are those of rlk_linear_logp_fwd.
+ *  - Scratch (error word and per-split partials) lives in a file-scope device
+ *    array of 32 MiB that every GPU which loads the library holds until the
+ *    process exits.  Sizes needing more than that (more than about 9400 rows
+ *    at V = 151936) are rejected with RLK_ERR_WORKSPACE_TOO_SMALL before
+ *    anything is enqueued.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current (cudaGetSymbolAddress); make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array: calls whose kernels overlap on the GPU
+ *    (for instance on two streams) race and corrupt each other's results.
+ *    Each call clears the error word itself; an out-of-range target gives NaN
+ *    logp for its row, and a timed-out internal wait turns all outputs NaN.
+ *  - Calls no allocation routine of CUDA or of any other library. */
+rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W,
+                                       const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                       float temperature, float* logp, float* entropy,
+                                       float* lse, void* stream);
+
 /* Self-check of the tensor-core mainloop shared by every kernel above:
  * C[M,N] fp32 = sum_k A[m,k] B[n,k] with bf16 inputs and fp32 accumulation.
  * a_mn_major == 0: A is stored [M,K] (K contiguous); != 0: stored [K,M].

@@ -207,3 +207,32 @@ class LinearLogp(torch.autograd.Function):
         dH, dW = rlk_linear_logp_bwd(hidden, W, targets, ctx.temperature, lse, entropy,
                                      dl.contiguous(), de.contiguous(), ctx.ws)
         return dH, dW.to(W.dtype), None, None
+
+
+_noalloc_fn = None
+
+
+def rlk_linear_logp_fwd_noalloc(hidden, W, targets, temperature, out=None, stream=None):
+    """Forward through the entry point that takes no workspace and allocates
+    nothing (its scratch is a fixed device array inside the library); for
+    callers that cannot allocate device memory.  Outputs as rlk_linear_logp_fwd."""
+    global _noalloc_fn
+    if _noalloc_fn is None:
+        f = lib().rlk_linear_logp_fwd_noalloc
+        f.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _P]
+        f.restype = ctypes.c_int
+        _noalloc_fn = f
+    _req(hidden, torch.bfloat16, "hidden", 2)
+    _req(W, torch.bfloat16, "W", 2)
+    _req(targets, torch.int64, "targets", 1)
+    T, H = hidden.shape
+    V = W.shape[0]
+    if W.shape[1] != H or targets.shape[0] != T:
+        raise ValueError("shape mismatch")
+    if out is None:
+        out = tuple(torch.empty(T, dtype=torch.float32, device=hidden.device) for _ in range(3))
+    logp, entropy, lse = out
+    _check(_noalloc_fn(_ptr(hidden), _ptr(W), _ptr(targets), T, H, V, float(temperature),
+                       _ptr(logp), _ptr(entropy), _ptr(lse), _stream(stream)),
+           "rlk_linear_logp_fwd_noalloc")
+    return logp, entropy, lse

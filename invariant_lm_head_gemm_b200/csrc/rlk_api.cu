@@ -413,3 +413,111 @@ const char* rlk_status_string(rlk_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward without a caller-provided workspace.
+//
+// For callers that cannot allocate device memory at all: code that runs
+// inside a host framework that owns every device byte (a serving engine with
+// a pre-reserved pool, a plugin host that forbids allocation calls), or that
+// cannot size a workspace ahead of time.  Their per-call scratch (the error
+// word and the forward's per-split partials) lives in one file-scope device
+// array that every GPU loading this library holds until the process exits.
+// ---------------------------------------------------------------------------
+namespace rlk {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t{32} << 20;  // 32 MiB per device
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch, looked up once per device with that
+// device current.  In host code the array's name is only a host-side stand-in.
+void* g_static_scratch_addr[kMaxDevices];
+
+rlk_status static_scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return RLK_ERR_UNSUPPORTED_DEVICE;
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return RLK_ERR_CUDA;
+    }
+    g_static_scratch_addr[dev] = p;
+  }
+  *out = g_static_scratch_addr[dev];
+  return RLK_OK;
+}
+
+// After a timed-out pipeline wait the outputs are not trustworthy; without a
+// caller-visible error word they are overwritten with NaN instead.
+__global__ void poison_on_timeout_kernel(const uint32_t* err, float* logp, float* entropy,
+                                         float* lse, int T) {
+  if ((*err & kDevErrTimeout) == 0) return;
+  const float nan = __int_as_float(0x7fc00000);
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+    logp[t] = nan;
+    entropy[t] = nan;
+    lse[t] = nan;
+  }
+}
+
+}  // namespace
+}  // namespace rlk
+
+extern "C" {
+
+
+rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W,
+                                       const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                       float temperature, float* logp, float* entropy,
+                                       float* lse, void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (T == 0) return RLK_OK;
+  if (!hidden || !W || !targets || !logp || !entropy || !lse) return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(targets, 8) || !aligned(logp, 4) ||
+      !aligned(entropy, 4) || !aligned(lse, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);
+  if (L.fwd_end > kStaticScratchBytes) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  void* scratch = nullptr;
+  if ((s = static_scratch_for_current_device(&scratch)) != RLK_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  // The array keeps the previous call's contents: only the error word must
+  // start at zero (every partial this call reads, it writes first).
+  if (cudaMemsetAsync(err, 0, kHeader, st) != cudaSuccess) return RLK_ERR_CUDA;
+  CUtensorMap mh, mw;
+  if (!map_kmajor(&mh, hidden, H, T, H, kBM) || !map_kmajor(&mw, W, H, V, H, kBN))
+    return RLK_ERR_CUDA;
+  Sched sc = make_sched(T, V, H, kFwdGroup);
+  EpiFwd::Params ep;
+  ep.targets = targets;
+  ep.part_m = reinterpret_cast<float*>(ws + L.pm);
+  ep.part_s = reinterpret_cast<float*>(ws + L.ps);
+  ep.part_b = reinterpret_cast<float*>(ws + L.pb);
+  ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
+  ep.T = static_cast<int>(T);
+  ep.V = static_cast<int>(V);
+  ep.scale_log2 = kLog2e / temperature;
+  if ((s = launch_gemm<EpiFwd, false, false>(mh, mw, sc, ep, err, st, sms)) != RLK_OK) return s;
+  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, st>>>(
+      ep.part_m, ep.part_s, ep.part_b, ep.ytgt, targets, static_cast<int>(T),
+      static_cast<int>(V), sc.num_groups, logp, entropy, lse, err);
+  poison_on_timeout_kernel<<<std::min<int64_t>(ceil_div(T, 256), 1024), 256, 0, st>>>(
+      err, logp, entropy, lse, static_cast<int>(T));
+  if (cudaGetLastError() != cudaSuccess) return RLK_ERR_CUDA;
+  return RLK_OK;
+}
+
+}  // extern "C"
