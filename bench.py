@@ -305,8 +305,7 @@ def run_ours(args):
     flops_tok = 8.0 * H * V
     step_tflops = flops_tok * T / (ms_max * 1e-3) / 1e12
     fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
-    nchunks = -(-V // 8192)
-    launches_per_step = 2 + 3 * nchunks
+    launches_per_step = 3      # forward GEMM, combine, fused backward
     value = world * T / (ms_max * 1e-3)
     line = {
         "metric": METRIC,

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include "rlk.h"
+#include "rlk_bwd.cuh"
 #include "rlk_gemm.cuh"
 
 namespace rlk {
@@ -40,9 +41,17 @@ int64_t fwd_groups(int64_t V) { return ceil_div(ceil_div(V, kBN), kFwdGroup); }
 // Vocab columns per backward chunk (a multiple of kBN, at most kVChunk).
 int64_t vchunk(int64_t V) { return std::min<int64_t>(kVChunk, ceil_div(V, kBN) * kBN); }
 
+// Plan of the fused backward for these sizes (see rlk_bwd.cuh).
+BwdPlan bwd_plan(int64_t T, int64_t H, int64_t V) { return make_bwd_plan(T, H, V, vchunk(V)); }
+
+size_t bwd_counter_words(const BwdPlan& p) {
+  const size_t nc = static_cast<size_t>(p.NC);
+  return nc * p.MT + nc * p.RT_full + nc * p.MT * p.NH + nc;
+}
+
 struct Layout {
   size_t pm, ps, pb, yt, fwd_end;
-  size_t dx, dh, bwd_end;
+  size_t dx[kDxBuffers], dh, cnt, bwd_end;
 };
 
 Layout layout(int64_t T, int64_t H, int64_t V) {
@@ -54,9 +63,12 @@ Layout layout(int64_t T, int64_t H, int64_t V) {
   L.pb = L.ps + align256(G * t * 4);
   L.yt = L.pb + align256(G * t * 4);
   L.fwd_end = L.yt + align256(t * 4);
-  L.dx = kHeader;
-  L.dh = L.dx + align256(t * static_cast<size_t>(vchunk(V)) * 2);
-  L.bwd_end = L.dh + align256(t * static_cast<size_t>(H) * 4);
+  const size_t dx_bytes = align256(t * static_cast<size_t>(vchunk(V)) * 2);
+  L.dx[0] = kHeader;
+  for (int i = 1; i < kDxBuffers; ++i) L.dx[i] = L.dx[i - 1] + dx_bytes;
+  L.dh = L.dx[kDxBuffers - 1] + dx_bytes;
+  L.cnt = L.dh + align256(t * static_cast<size_t>(H) * 4);
+  L.bwd_end = L.cnt + align256(bwd_counter_words(bwd_plan(T, H, V)) * 4);
   return L;
 }
 
@@ -265,72 +277,58 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   if ((s = check_device(&sms)) != RLK_OK) return s;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
-  __nv_bfloat16* dX = reinterpret_cast<__nv_bfloat16*>(ws + L.dx);
-  float* dh_acc = reinterpret_cast<float*>(ws + L.dh);
-  const int64_t ldx = vchunk(V);
-  const int64_t nchunks = ceil_div(V, ldx);
-
-  CUtensorMap m_hid_k, m_w_k, m_w_mn, m_hid_mn;
-  if (!map_kmajor(&m_hid_k, hidden, H, T, H, kBM) || !map_kmajor(&m_w_k, W, H, V, H, kBN) ||
-      !map_mnmajor(&m_w_mn, W, H, V, H) || !map_mnmajor(&m_hid_mn, hidden, H, T, H))
+  BwdParams P;
+  P.plan = bwd_plan(T, H, V);
+  const BwdPlan& pl = P.plan;
+  if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
+      !map_kmajor(&P.maps.w_k, W, H, V, H, kBN) || !map_mnmajor(&P.maps.w_mn, W, H, V, H) ||
+      !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
     return RLK_ERR_CUDA;
-
-  for (int64_t c = 0; c < nchunks; ++c) {
-    const int64_t c0 = c * ldx;
-    const int64_t valid = std::min(ldx, V - c0);
-
-    // (1) recompute the chunk's logits and write its bf16 dlogits to dX.
-    Sched s1 = make_sched(T, valid, H, 1);
-    s1.b_n_off = static_cast<int>(c0);
-    s1.b_mn_extent = static_cast<int>(V);
-    EpiDlogits::Params p1;
-    p1.targets = targets;
-    p1.lse = lse;
-    p1.entropy = entropy;
-    p1.dlogp = dlogp;
-    p1.dentropy = dentropy;
-    p1.dX = dX;
-    p1.err = err;
-    p1.T = static_cast<int>(T);
-    p1.V = static_cast<int>(V);
-    p1.c0 = static_cast<int>(c0);
-    p1.ldx = static_cast<int>(ldx);
-    p1.scale_log2 = kLog2e / temperature;
-    p1.inv_tau = 1.0f / temperature;
-    if ((s = launch_gemm<EpiDlogits, false, false>(m_hid_k, m_w_k, s1, p1, err, st, sms)) !=
-        RLK_OK)
-      return s;
-
-    CUtensorMap m_dx_k, m_dx_mn;
-    if (!map_kmajor(&m_dx_k, dX, valid, T, ldx, kBM) || !map_mnmajor(&m_dx_mn, dX, valid, T, ldx))
+  for (int i = 0; i < kDxBuffers; ++i) {
+    P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
+    if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
+        !map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx))
       return RLK_ERR_CUDA;
+  }
+  P.targets = targets;
+  P.lse = lse;
+  P.entropy = entropy;
+  P.dlogp = dlogp;
+  P.dentropy = dentropy;
+  P.dh_acc = reinterpret_cast<float*>(ws + L.dh);
+  P.dhidden = reinterpret_cast<__nv_bfloat16*>(dHidden);
+  P.dW = dW;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  const size_t nc = static_cast<size_t>(pl.NC);
+  P.rdone_m = cnt;
+  P.rdone_j = P.rdone_m + nc * pl.MT;
+  P.hdone = P.rdone_j + nc * pl.RT_full;
+  P.bufdone = P.hdone + nc * pl.MT * pl.NH;
+  P.err = reinterpret_cast<uint32_t*>(ws);
+  P.scale_log2 = kLog2e / temperature;
+  P.inv_tau = 1.0f / temperature;
 
-    // (2) dHidden += dX[T, valid] . W[c0 : c0 + valid, :]
-    Sched s2 = make_sched(T, H, valid, 1);
-    s2.b_k_off = static_cast<int>(c0);
-    EpiDh::Params p2;
-    p2.acc = dh_acc;
-    p2.out = reinterpret_cast<__nv_bfloat16*>(dHidden);
-    p2.T = static_cast<int>(T);
-    p2.H = static_cast<int>(H);
-    p2.mode = nchunks == 1 ? EpiDh::kOnly
-              : c == 0     ? EpiDh::kFirst
-              : c == nchunks - 1 ? EpiDh::kLast
-                                 : EpiDh::kMiddle;
-    if ((s = launch_gemm<EpiDh, false, true>(m_dx_k, m_w_mn, s2, p2, err, st, sms)) != RLK_OK)
-      return s;
-
-    // (3) dW[c0 : c0 + valid, :] = dX[T, valid]^T . hidden[T, H]
-    Sched s3 = make_sched(valid, H, T, 1);
-    EpiStore::Params p3;
-    p3.out = dW + static_cast<size_t>(c0) * H;
-    p3.rows = static_cast<int>(valid);
-    p3.ncols = static_cast<int>(H);
-    p3.ld = static_cast<int>(H);
-    if ((s = launch_gemm<EpiStore, true, true>(m_dx_mn, m_hid_mn, s3, p3, err, st, sms)) !=
-        RLK_OK)
-      return s;
+  if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
+  if (cudaFuncSetAttribute(bwd_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemBytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  // Units wait on units of other CTAs, so every CTA must be resident: the
+  // launch is cooperative (at most one CTA per SM fits anyway).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>(pl.total, sms)));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, bwd_fused_kernel, P) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
   }
   g_calls[1].fetch_add(1);
   return RLK_OK;

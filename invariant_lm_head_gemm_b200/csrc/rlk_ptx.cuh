@@ -198,3 +198,44 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 }  // namespace rlk
+
+namespace rlk {
+
+// ---------------------------------------------------------------- cross-CTA signalling
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Orders this thread's generic-proxy global accesses with its later (or
+// earlier) async-proxy ones, e.g. a TMA load of data another CTA stored.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Named barrier 1 over the 128 epilogue threads.
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Waits until *p >= target (acquire).  Bounded like mbar_wait_bounded.
+__device__ __forceinline__ bool wait_counter_bounded(const uint32_t* p, uint32_t target,
+                                                     volatile int* abort_flag, uint32_t* err) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) >= target) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(err, kDevErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+}  // namespace rlk

@@ -42,13 +42,16 @@ def test_workspace_bytes(L):
     def a(x):
         return (x + 255) // 256 * 256
     assert fwd == 256 + 3 * a(297 * T * 4) + a(T * 4)
-    # bwd: header + [T, 8192] bf16 dlogits chunk + [T, H] fp32 dHidden accumulator
-    assert both == max(fwd, 256 + a(T * 8192 * 2) + a(T * H * 4))
+    # bwd: header + 3 x [T, 8192] bf16 dlogits chunk buffers + [T, H] fp32 dHidden
+    # accumulator + the fused backward's dependency counters
+    NC, MT, NH, RT = 19, (T + 127) // 128, H // 256, 8192 // 256
+    counters = NC * MT + NC * RT + NC * MT * NH + NC
+    assert both == max(fwd, 256 + 3 * a(T * 8192 * 2) + a(T * H * 4) + a(counters * 4))
     assert binding.workspace_bytes(4, 100, 10) == 0          # H % 64 != 0
     assert binding.workspace_bytes(4, 64, 0) == 0
     assert binding.workspace_bytes(0, 64, 10) > 0
     # small V: the chunk buffer shrinks to V rounded up to 256 columns
-    assert binding.workspace_bytes(8, 64, 300, True) >= 256 + 8 * 512 * 2 + 8 * 64 * 4
+    assert binding.workspace_bytes(8, 64, 300, True) >= 256 + 3 * 8 * 512 * 2 + 8 * 64 * 4
 
 
 A16 = 0x10000        # fake, never dereferenced: validation must fail first
