@@ -11,8 +11,7 @@
 #include <cuda_runtime.h>
 
 #include "rlk.h"
-#include "rlk_bwd.cuh"
-#include "rlk_gemm.cuh"
+#include "rlk_kernel.cuh"
 
 namespace rlk {
 namespace {
@@ -46,7 +45,7 @@ BwdPlan bwd_plan(int64_t T, int64_t H, int64_t V) { return make_bwd_plan(T, H, V
 
 size_t bwd_counter_words(const BwdPlan& p) {
   const size_t nc = static_cast<size_t>(p.NC);
-  return nc * p.MT + nc * p.RT_full + nc * p.MT * p.NH + nc;
+  return nc * p.MT + nc * p.RT_full + nc * p.MT * p.NH + nc + 1;
 }
 
 struct Layout {
@@ -80,6 +79,8 @@ rlk_status check_sizes(int64_t T, int64_t H, int64_t V, float temperature) {
   if (!std::isfinite(kLog2e / temperature)) return RLK_ERR_INVALID_ARG;
   if (H % 64 != 0 || H > (int64_t{1} << 20)) return RLK_ERR_UNSUPPORTED_SHAPE;
   if (V >= (int64_t{1} << 31) || T >= (int64_t{1} << 31)) return RLK_ERR_UNSUPPORTED_SHAPE;
+  // unit indices of the backward travel as 32-bit integers
+  if (make_bwd_plan(T, H, V, vchunk(V)).total >= (int64_t{1} << 31)) return RLK_ERR_UNSUPPORTED_SHAPE;
   return RLK_OK;
 }
 
@@ -136,7 +137,8 @@ EncodeTiledFn encode_fn() {
 // elements per row, `outer` rows and a row pitch of `pitch_elems`; boxes of
 // box_inner x box_outer, 128-byte swizzle, zero fill outside the matrix.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -144,8 +146,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // K-major operand [rows, K] (K contiguous): one 64 x box_rows box per stage.
@@ -159,33 +161,88 @@ bool map_mnmajor(CUtensorMap* m, const void* base, int64_t MN, int64_t K, int64_
   return make_map(m, base, MN, K, pitch, 64, 64);
 }
 
-Sched make_sched(int64_t M, int64_t N, int64_t K, int group) {
-  Sched s;
-  s.num_m_tiles = static_cast<int>(ceil_div(M, kBM));
-  s.num_n_tiles = static_cast<int>(ceil_div(N, kBN));
-  s.group = group;
-  s.num_groups = static_cast<int>(ceil_div(s.num_n_tiles, group));
-  s.num_units = s.num_m_tiles * s.num_groups;
-  s.num_k_blocks = static_cast<int>(ceil_div(K, kBK));
-  s.a_m_off = s.a_k_off = s.b_n_off = s.b_k_off = 0;
-  s.a_mn_extent = static_cast<int>(M);
-  s.b_mn_extent = static_cast<int>(N);
-  return s;
-}
+int g_max_clusters[3][kMaxDevices];
 
-template <class Epi, bool A_MN, bool B_MN>
-rlk_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const Sched& sc,
-                       const typename Epi::Params& ep, uint32_t* err, cudaStream_t st,
-                       int num_sms) {
-  if (sc.num_units <= 0) return RLK_OK;
-  auto kern = gemm_kernel<Epi, A_MN, B_MN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes)) != cudaSuccess) {
+// Launches pair_kernel<Mode> on clusters of two CTAs: at most one cluster per
+// unit and no more clusters than can be resident at once.  `cooperative`
+// makes the launch fail rather than start with some CTAs not resident (the
+// backward's units wait on each other).
+template <int Mode>
+rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long total,
+                       bool cooperative, cudaStream_t st) {
+  if (total <= 0) return RLK_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return RLK_ERR_CUDA;
   }
-  const int grid = std::min(sc.num_units, num_sms);
-  kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, sc, ep, err);
+  auto kern = pair_kernel<Mode>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kPSmemBytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int& mc = g_max_clusters[Mode][dev];
+  if (mc == 0) {
+    cfg.gridDim = dim3(2);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return RLK_ERR_CUDA;
+    }
+    mc = n;
+  }
+  cfg.numAttrs = cooperative ? 2 : 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<long long>(total, mc)));
+  if (cudaLaunchKernelEx(&cfg, kern, args) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  return RLK_OK;
+}
+
+// Forward: pair-tile GEMM with the online epilogue, then the combine.
+rlk_status enqueue_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                       int64_t T, int64_t H, int64_t V, float temperature, float* logp,
+                       float* entropy, float* lse, uint8_t* ws, const Layout& L,
+                       cudaStream_t st) {
+  FwdArgs a;
+  if (!map_kmajor(&a.hid_k, hidden, H, T, H, kBM) || !map_kmajor(&a.w_k, W, H, V, H, kBM))
+    return RLK_ERR_CUDA;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  a.ep.targets = targets;
+  a.ep.part_m = reinterpret_cast<float*>(ws + L.pm);
+  a.ep.part_s = reinterpret_cast<float*>(ws + L.ps);
+  a.ep.part_b = reinterpret_cast<float*>(ws + L.pb);
+  a.ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
+  a.ep.T = static_cast<int>(T);
+  a.ep.V = static_cast<int>(V);
+  a.ep.scale_log2 = kLog2e / temperature;
+  a.err = err;
+  a.MT = static_cast<int>(ceil_div(T, kPairM));
+  a.NT = static_cast<int>(ceil_div(V, kBN));
+  a.group = kFwdGroup;
+  a.NG = static_cast<int>(fwd_groups(V));
+  a.KB = static_cast<int>(H / kBK);
+  a.total = static_cast<long long>(a.MT) * a.NG;
+  rlk_status s = launch_pair<kModeFwd>(a, a.total, false, st);
+  if (s != RLK_OK) return s;
+  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, st>>>(
+      a.ep.part_m, a.ep.part_s, a.ep.part_b, a.ep.ytgt, targets, static_cast<int>(T),
+      static_cast<int>(V), a.NG, logp, entropy, lse, err);
   return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
 }
 
@@ -220,29 +277,9 @@ rlk_status rlk_linear_logp_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   if ((s = check_device(&sms)) != RLK_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
-  CUtensorMap mh, mw;
-  if (!map_kmajor(&mh, hidden, H, T, H, kBM) || !map_kmajor(&mw, W, H, V, H, kBN))
-    return RLK_ERR_CUDA;
-
-  Sched sc = make_sched(T, V, H, kFwdGroup);
-  EpiFwd::Params ep;
-  ep.targets = targets;
-  ep.part_m = reinterpret_cast<float*>(ws + L.pm);
-  ep.part_s = reinterpret_cast<float*>(ws + L.ps);
-  ep.part_b = reinterpret_cast<float*>(ws + L.pb);
-  ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
-  ep.T = static_cast<int>(T);
-  ep.V = static_cast<int>(V);
-  ep.scale_log2 = kLog2e / temperature;
-  if ((s = launch_gemm<EpiFwd, false, false>(mh, mw, sc, ep, err, st, sms)) != RLK_OK) return s;
-
-  const int G = sc.num_groups;
-  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, st>>>(
-      ep.part_m, ep.part_s, ep.part_b, ep.ytgt, targets, static_cast<int>(T),
-      static_cast<int>(V), G, logp, entropy, lse, err);
-  if (cudaGetLastError() != cudaSuccess) return RLK_ERR_CUDA;
+  s = enqueue_fwd(hidden, W, targets, T, H, V, temperature, logp, entropy, lse,
+                  static_cast<uint8_t*>(workspace), L, st);
+  if (s != RLK_OK) return s;
   g_calls[0].fetch_add(1);
   return RLK_OK;
 }
@@ -281,13 +318,14 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   P.plan = bwd_plan(T, H, V);
   const BwdPlan& pl = P.plan;
   if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
-      !map_kmajor(&P.maps.w_k, W, H, V, H, kBN) || !map_mnmajor(&P.maps.w_mn, W, H, V, H) ||
+      !map_kmajor(&P.maps.w_k, W, H, V, H, kBM) || !map_mnmajor(&P.maps.w_mn, W, H, V, H) ||
       !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
     return RLK_ERR_CUDA;
   for (int i = 0; i < kDxBuffers; ++i) {
     P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
     if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx))
+        !map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx) ||
+        !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
       return RLK_ERR_CUDA;
   }
   P.targets = targets;
@@ -304,32 +342,14 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   P.rdone_j = P.rdone_m + nc * pl.MT;
   P.hdone = P.rdone_j + nc * pl.RT_full;
   P.bufdone = P.hdone + nc * pl.MT * pl.NH;
+  P.next_unit = P.bufdone + nc;
   P.err = reinterpret_cast<uint32_t*>(ws);
   P.scale_log2 = kLog2e / temperature;
   P.inv_tau = 1.0f / temperature;
 
   if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
-  if (cudaFuncSetAttribute(bwd_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes)) != cudaSuccess) {
-    cudaGetLastError();
-    return RLK_ERR_CUDA;
-  }
-  // Units wait on units of other CTAs, so every CTA must be resident: the
-  // launch is cooperative (at most one CTA per SM fits anyway).
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(std::min<long long>(pl.total, sms)));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, bwd_fused_kernel, P) != cudaSuccess) {
-    cudaGetLastError();
-    return RLK_ERR_CUDA;
-  }
+  // Units wait on units of other CTAs, so every CTA must be resident.
+  if ((s = launch_pair<kModeBwd>(P, pl.total, true, st)) != RLK_OK) return s;
   g_calls[1].fetch_add(1);
   return RLK_OK;
 }
@@ -353,24 +373,24 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(workspace);
 
-  CUtensorMap ma, mb;
-  bool ok = a_mn_major ? map_mnmajor(&ma, A, M, K, M) : map_kmajor(&ma, A, K, M, K, kBM);
-  ok = ok && (b_mn_major ? map_mnmajor(&mb, B, N, K, N) : map_kmajor(&mb, B, K, N, K, kBN));
+  GemmArgs a;
+  bool ok = a_mn_major ? map_mnmajor(&a.a, A, M, K, M) : map_kmajor(&a.a, A, K, M, K, kBM);
+  ok = ok && (b_mn_major ? map_mnmajor(&a.b, B, N, K, N) : map_kmajor(&a.b, B, K, N, K, kBM));
   if (!ok) return RLK_ERR_CUDA;
-  Sched sc = make_sched(M, N, K, 1);
-  EpiStore::Params ep;
-  ep.out = C;
-  ep.rows = static_cast<int>(M);
-  ep.ncols = static_cast<int>(N);
-  ep.ld = static_cast<int>(N);
-  if (!a_mn_major && !b_mn_major)
-    s = launch_gemm<EpiStore, false, false>(ma, mb, sc, ep, err, st, sms);
-  else if (!a_mn_major && b_mn_major)
-    s = launch_gemm<EpiStore, false, true>(ma, mb, sc, ep, err, st, sms);
-  else if (a_mn_major && !b_mn_major)
-    s = launch_gemm<EpiStore, true, false>(ma, mb, sc, ep, err, st, sms);
-  else
-    s = launch_gemm<EpiStore, true, true>(ma, mb, sc, ep, err, st, sms);
+  a.ep.out = C;
+  a.ep.rows = static_cast<int>(M);
+  a.ep.ncols = static_cast<int>(N);
+  a.ep.ld = static_cast<int>(N);
+  a.err = err;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.MT = static_cast<int>(ceil_div(M, kPairM));
+  a.NT = static_cast<int>(ceil_div(N, kBN));
+  a.KB = static_cast<int>(ceil_div(K, kBK));
+  a.a_mn = a_mn_major ? 1 : 0;
+  a.b_mn = b_mn_major ? 1 : 0;
+  a.total = static_cast<long long>(a.MT) * a.NT;
+  s = launch_pair<kModeGemm>(a, a.total, false, st);
   if (s == RLK_OK) g_calls[2].fetch_add(1);
   return s;
 }
@@ -495,23 +515,9 @@ rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W
   // The array keeps the previous call's contents: only the error word must
   // start at zero (every partial this call reads, it writes first).
   if (cudaMemsetAsync(err, 0, kHeader, st) != cudaSuccess) return RLK_ERR_CUDA;
-  CUtensorMap mh, mw;
-  if (!map_kmajor(&mh, hidden, H, T, H, kBM) || !map_kmajor(&mw, W, H, V, H, kBN))
-    return RLK_ERR_CUDA;
-  Sched sc = make_sched(T, V, H, kFwdGroup);
-  EpiFwd::Params ep;
-  ep.targets = targets;
-  ep.part_m = reinterpret_cast<float*>(ws + L.pm);
-  ep.part_s = reinterpret_cast<float*>(ws + L.ps);
-  ep.part_b = reinterpret_cast<float*>(ws + L.pb);
-  ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
-  ep.T = static_cast<int>(T);
-  ep.V = static_cast<int>(V);
-  ep.scale_log2 = kLog2e / temperature;
-  if ((s = launch_gemm<EpiFwd, false, false>(mh, mw, sc, ep, err, st, sms)) != RLK_OK) return s;
-  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, st>>>(
-      ep.part_m, ep.part_s, ep.part_b, ep.ytgt, targets, static_cast<int>(T),
-      static_cast<int>(V), sc.num_groups, logp, entropy, lse, err);
+  if ((s = enqueue_fwd(hidden, W, targets, T, H, V, temperature, logp, entropy, lse, ws, L, st)) !=
+      RLK_OK)
+    return s;
   poison_on_timeout_kernel<<<std::min<int64_t>(ceil_div(T, 256), 1024), 256, 0, st>>>(
       err, logp, entropy, lse, static_cast<int>(T));
   if (cudaGetLastError() != cudaSuccess) return RLK_ERR_CUDA;

@@ -34,7 +34,8 @@
 
 namespace rlk {
 
-constexpr int kBM = 128;
+constexpr int kBM = 128;     // accumulator rows per CTA
+constexpr int kPairM = 256;  // accumulator rows per CTA pair
 constexpr int kBN = 256;
 constexpr int kBK = 64;
 constexpr int kStages = 4;
@@ -215,7 +216,15 @@ struct EpiDlogits {
     }
   }
 
-  __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt) {
+  // One 128 x 256 tile, 32 columns at a time.  Each warp stages its 32 x 32
+  // bf16 block in shared memory (two 2 KB buffers, `stage`) and one lane
+  // writes it to dX[warp_row0 .. +32, col .. +32] with a TMA store (rows past
+  // T are not written).  The caller waits for the stores (bulk_wait_all)
+  // before publishing the tile.
+  __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt,
+                              const CUtensorMap* store_map, uint32_t stage, int lane,
+                              int warp_row0) {
+    const bool any_row = warp_row0 < p.T;
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
       uint32_t r[32];
@@ -239,16 +248,22 @@ struct EpiDlogits {
 #pragma unroll
         for (int j = 0; j < 32; ++j) dx[j] = (j == d) ? dx[j] + st.hot : dx[j];
       }
-      if (st.valid) {
-        uint4* dst = reinterpret_cast<uint4*>(p.dX + static_cast<size_t>(st.row) * p.ldx + loc0);
+      if (any_row) {
+        const uint32_t buf = stage + (c & 1) * 2048u;
+        if (lane == 0) bulk_wait_read_le1();  // the store two chunks back has read `buf`
+        __syncwarp();
+        const uint32_t row_addr = buf + lane * 64u;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 w;
-          w.x = pack_bf16x2(dx[8 * q + 0], dx[8 * q + 1]);
-          w.y = pack_bf16x2(dx[8 * q + 2], dx[8 * q + 3]);
-          w.z = pack_bf16x2(dx[8 * q + 4], dx[8 * q + 5]);
-          w.w = pack_bf16x2(dx[8 * q + 6], dx[8 * q + 7]);
-          dst[q] = w;
+        for (int q = 0; q < 4; ++q)
+          st_shared_v4(row_addr + q * 16u, pack_bf16x2(dx[8 * q + 0], dx[8 * q + 1]),
+                       pack_bf16x2(dx[8 * q + 2], dx[8 * q + 3]),
+                       pack_bf16x2(dx[8 * q + 4], dx[8 * q + 5]),
+                       pack_bf16x2(dx[8 * q + 6], dx[8 * q + 7]));
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(store_map, buf, loc0, warp_row0);
+          bulk_commit_group();
         }
       }
     }

@@ -1,0 +1,572 @@
+// rlk_kernel.cuh -- the persistent CTA-pair kernel behind the forward pass,
+// the backward pass and the self-check GEMM.
+//
+// Each cluster of two CTAs computes 256 x 256 fp32 accumulator tiles with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): CTA r of the pair
+// loads rows [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128)
+// of the B tile (its half of N) into its own shared memory, the pair's leader
+// (rank 0) issues the MMAs, and each CTA's TMEM receives its 128 accumulator
+// rows.  Per CTA and 64-wide K block that is 16 KB of A and 16 KB of B, so a
+// six-stage TMA ring fits in shared memory and covers about 2.5k MMA cycles
+// of load latency.
+//
+// Roles per CTA (192 threads): warp 0 TMA producer (both CTAs load; the
+// leader arms its "full" barrier with both CTAs' bytes and both CTAs' loads
+// complete on it); warp 1 allocates the pair's TMEM (two 256-column
+// accumulators) and, in the leader, issues the MMAs and commits them to the
+// "empty" / "full accumulator" barriers of both CTAs; warps 2-5 epilogue,
+// one accumulator row per thread, releasing the accumulator to the leader.
+//
+// Units are walked in ascending order, pair p taking units p, p + pairs, ...;
+// a unit is `ntiles` consecutive N tiles of one M tile (several only in the
+// forward, whose epilogue carries its online reduction across them).  Every
+// wait is time-bounded; on expiry the kernel records RLK_DEVERR_TIMEOUT,
+// drains its in-flight copies and MMAs and returns.
+#pragma once
+
+#include "rlk_bwd.cuh"
+#include "rlk_gemm.cuh"
+
+namespace rlk {
+
+constexpr int kPStages = 6;
+constexpr uint32_t kPAStage = kBM * kBK * 2;  // this CTA's 128 rows of A: 16 KB
+constexpr uint32_t kPBStage = kBM * kBK * 2;  // this CTA's 128 rows of B: 16 KB
+constexpr uint32_t kPStaging = 4 * 4096;     // per epilogue warp: two 2 KB store buffers
+constexpr int kRing = 4;                      // units in flight through the pair's broadcast ring
+constexpr int kPNumBars = 2 * kPStages + 5 + 2 * kRing;
+constexpr size_t kPSmemBytes =
+    1024 + kPStages * (kPAStage + kPBStage) + kPStaging + kPNumBars * 8 + 64;
+
+enum : int { kModeFwd = 0, kModeBwd = 1, kModeGemm = 2 };
+enum : int { kJobFwd = 3, kJobGemm = 4 };  // backward jobs use kUnitR / kUnitH / kUnitD
+
+struct FwdArgs {
+  CUtensorMap hid_k;  // hidden [T,H], box 64 x 128
+  CUtensorMap w_k;    // W [V,H], box 64 x 128
+  EpiFwd::Params ep;
+  uint32_t* err;
+  int MT;             // 256-row M tiles
+  int NT;             // 256-column vocab tiles
+  int group;          // vocab tiles per unit
+  int NG;             // vocab splits = ceil(NT / group)
+  int KB;             // K blocks (H / 64)
+  long long total;    // MT * NG
+};
+
+struct GemmArgs {
+  CUtensorMap a;      // K-major box 64 x 128, or MN-major box 64 x 64
+  CUtensorMap b;
+  EpiStore::Params ep;
+  uint32_t* err;
+  int M, N, MT, NT, KB;
+  int a_mn, b_mn;
+  long long total;
+};
+
+template <int Mode>
+struct ModeArgs;
+template <>
+struct ModeArgs<kModeFwd> {
+  using type = FwdArgs;
+};
+template <>
+struct ModeArgs<kModeBwd> {
+  using type = BwdParams;
+};
+template <>
+struct ModeArgs<kModeGemm> {
+  using type = GemmArgs;
+};
+
+// What one unit loads and computes.
+struct Job {
+  int type;
+  int c;            // vocab chunk (backward)
+  int mt;           // M tile (256 rows)
+  int nt;           // first N tile (256 columns)
+  int ntiles;       // N tiles in the unit
+  int kbs;          // K blocks per tile
+  bool a_mn, b_mn;  // operand majorness
+  const CUtensorMap* mA;
+  const CUtensorMap* mB;
+  int a_row0;       // M coordinate of the tile's first row in A's tensor map
+  int b_col0;       // N coordinate of the first tile's first column in B's map
+  int bk0;          // K offset of B's map
+  int a_ext;        // M extent of A's map: boxes starting at or past it are skipped
+  int b_ext;        // N extent of B's map
+};
+
+__device__ __forceinline__ Job make_job(const FwdArgs& P, long long u) {
+  Job j;
+  j.type = kJobFwd;
+  j.c = 0;
+  j.mt = static_cast<int>(u % P.MT);
+  const int g = static_cast<int>(u / P.MT);
+  j.nt = g * P.group;
+  j.ntiles = min(P.group, P.NT - j.nt);
+  j.kbs = P.KB;
+  j.a_mn = j.b_mn = false;
+  j.mA = &P.hid_k;
+  j.mB = &P.w_k;
+  j.a_row0 = j.mt * kPairM;
+  j.b_col0 = j.nt * kBN;
+  j.bk0 = 0;
+  j.a_ext = P.ep.T;
+  j.b_ext = P.ep.V;
+  return j;
+}
+
+__device__ __forceinline__ Job make_job(const GemmArgs& P, long long u) {
+  Job j;
+  j.type = kJobGemm;
+  j.c = 0;
+  j.mt = static_cast<int>(u % P.MT);
+  j.nt = static_cast<int>(u / P.MT);
+  j.ntiles = 1;
+  j.kbs = P.KB;
+  j.a_mn = P.a_mn != 0;
+  j.b_mn = P.b_mn != 0;
+  j.mA = &P.a;
+  j.mB = &P.b;
+  j.a_row0 = j.mt * kPairM;
+  j.b_col0 = j.nt * kBN;
+  j.bk0 = 0;
+  j.a_ext = P.M;
+  j.b_ext = P.N;
+  return j;
+}
+
+__device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
+  const BwdPlan& pl = P.plan;
+  const BwdUnit un = bwd_decode(pl, u);
+  Job j;
+  j.type = un.type;
+  j.c = un.c;
+  j.mt = un.a;
+  j.nt = un.b;
+  j.ntiles = 1;
+  j.bk0 = 0;
+  const int buf = un.c % kDxBuffers;
+  if (un.type == kUnitR) {
+    j.kbs = pl.KB_R;
+    j.a_mn = j.b_mn = false;
+    j.mA = &P.maps.hid_k;
+    j.mB = &P.maps.w_k;
+    j.a_row0 = un.a * kPairM;
+    j.b_col0 = un.c * pl.ldx + un.b * kBN;
+    j.a_ext = pl.T;
+    j.b_ext = pl.V;
+  } else if (un.type == kUnitH) {
+    j.kbs = (bwd_chunk_valid(pl, un.c) + kBK - 1) / kBK;
+    j.a_mn = false;
+    j.b_mn = true;
+    j.mA = &P.maps.dx_k[buf];
+    j.mB = &P.maps.w_mn;
+    j.a_row0 = un.a * kPairM;
+    j.b_col0 = un.b * kBN;
+    j.bk0 = un.c * pl.ldx;
+    j.a_ext = pl.T;
+    j.b_ext = pl.H;
+  } else {
+    j.kbs = pl.KB_D;
+    j.a_mn = j.b_mn = true;
+    j.mA = &P.maps.dx_mn[buf];
+    j.mB = &P.maps.hid_mn;
+    j.a_row0 = un.a * kPairM;
+    j.b_col0 = un.b * kBN;
+    j.a_ext = pl.ldx;
+    j.b_ext = pl.H;
+  }
+  return j;
+}
+
+__device__ __forceinline__ long long total_units(const FwdArgs& P) { return P.total; }
+__device__ __forceinline__ long long total_units(const GemmArgs& P) { return P.total; }
+__device__ __forceinline__ long long total_units(const BwdParams& P) { return P.plan.total; }
+__device__ __forceinline__ uint32_t* err_word(const FwdArgs& P) { return P.err; }
+__device__ __forceinline__ uint32_t* err_word(const GemmArgs& P) { return P.err; }
+__device__ __forceinline__ uint32_t* err_word(const BwdParams& P) { return P.err; }
+
+// Bytes CTA `rank` loads per K block of tile `t` of the job.
+__device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank) {
+  uint32_t bytes = 0;
+  const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
+  if (!j.a_mn) {
+    if (a0 < j.a_ext) bytes += kPAStage;
+  } else {
+    if (a0 < j.a_ext) bytes += kBox;
+    if (a0 + 64 < j.a_ext) bytes += kBox;
+  }
+  const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
+  if (!j.b_mn) {
+    if (b0 < j.b_ext) bytes += kPBStage;
+  } else {
+    if (b0 < j.b_ext) bytes += kBox;
+    if (b0 + 64 < j.b_ext) bytes += kBox;
+  }
+  return bytes;
+}
+
+template <int Mode>
+__global__ void __launch_bounds__(kThreads, 1)
+    pair_kernel(const __grid_constant__ typename ModeArgs<Mode>::type P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + kPStages * kPAStage;
+  const uint32_t sStage = sB + kPStages * kPBStage;
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(smem + kPStages * (kPAStage + kPBStage) + kPStaging);
+  const uint32_t bar0 = smem_u32(bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kPNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ep_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* ep_unit = reinterpret_cast<volatile int*>(tmem_slot + 3);
+  const uint32_t ring_addr = smem_u32(tmem_slot + 4);  // kRing unit indices
+
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kPStages + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kPStages + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kPStages + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kPStages + 4);
+  auto sfull_bar = [&](int i) { return bar0 + 8u * (2 * kPStages + 5 + i); };
+  auto sempty_bar = [&](int i) { return bar0 + 8u * (2 * kPStages + 5 + kRing + i); };
+
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const long long pair = blockIdx.x >> 1;
+  const long long npairs = gridDim.x >> 1;
+  const long long total = total_units(P);
+  uint32_t* err = err_word(P);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 8);  // one arrival per epilogue warp of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(sfull_bar(i), 1);
+      mbar_init(sempty_bar(i), 4);  // leader MMA + both CTAs' epilogues + the peer's producer
+    }
+    *abort_flag = 0;
+    *ep_ok = 1;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before anything signals them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // Unit order.  Forward and self-check GEMM: pair p runs units p, p + pairs,
+  // ...  Backward (units of unequal length that wait on each other): the
+  // leader's producer claims the next unit from a global counter, in
+  // ascending order, and broadcasts it through a kRing-slot ring to the
+  // leader's MMA issuer, the peer's producer and both CTAs' epilogues.
+  constexpr bool kDynamic = Mode == kModeBwd;
+  auto static_unit = [&](uint32_t k) -> long long {
+    const long long u = pair + static_cast<long long>(k) * npairs;
+    return u < total ? u : -1;
+  };
+  auto fetch_unit = [&](uint32_t k) -> long long {
+    const int slot = k % kRing;
+    if (!mbar_wait_cluster_bounded(sfull_bar(slot), (k / kRing) & 1u, abort_flag, err)) return -1;
+    const int v = static_cast<int>(ld_shared_u32(ring_addr + 4u * slot));
+    mbar_arrive_cluster(mapa_shared(sempty_bar(slot), 0));
+    return v;
+  };
+  auto claim_unit = [&](uint32_t k) -> long long {
+    const int slot = k % kRing;
+    if (!mbar_wait_bounded(sempty_bar(slot), ((k / kRing) & 1u) ^ 1u, abort_flag, err)) return -1;
+    long long u = -1;
+    if constexpr (kDynamic) u = atomicAdd(P.next_unit, 1u);
+    if (u >= total) u = -1;
+    st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 0), static_cast<uint32_t>(u));
+    st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 1), static_cast<uint32_t>(u));
+    mbar_arrive_cluster(mapa_shared(sfull_bar(slot), 0));
+    mbar_arrive_cluster(mapa_shared(sfull_bar(slot), 1));
+    return u;
+  };
+
+  uint32_t issued = 0;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        long long u;
+        if constexpr (kDynamic) {
+          u = leader ? claim_unit(k) : fetch_unit(k);
+        } else {
+          u = static_unit(k);
+        }
+        if (u < 0) break;
+        const Job j = make_job(P, u);
+        if (j.type < 0) break;
+        if constexpr (Mode == kModeBwd) {
+          const BwdPlan& pl = P.plan;
+          if (j.type == kUnitH) {
+            ok = wait_counter_bounded(P.rdone_m + static_cast<size_t>(j.c) * pl.MT + j.mt,
+                                      2u * static_cast<uint32_t>(bwd_rt(pl, j.c)), abort_flag,
+                                      err);
+          } else if (j.type == kUnitD) {
+            ok = wait_counter_bounded(P.rdone_j + static_cast<size_t>(j.c) * pl.RT_full + j.mt,
+                                      2u * static_cast<uint32_t>(pl.MT), abort_flag, err);
+          }
+          if (!ok) break;
+          if (j.type != kUnitR) fence_proxy_async_global();
+        }
+        if (k == 0) {
+          tma_prefetch_desc(j.mA);
+          tma_prefetch_desc(j.mB);
+        }
+        for (int t = 0; ok && t < j.ntiles; ++t) {
+          const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
+          const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
+          const uint32_t bytes_all = leader ? job_bytes(j, t, 0) + job_bytes(j, t, 1) : 0u;
+          for (int kb = 0; kb < j.kbs; ++kb) {
+            const int s = issued % kPStages;
+            const uint32_t ph = (issued / kPStages) & 1u;
+            if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = mapa_shared(full_bar(s), 0);
+            if (leader) mbar_arrive_expect_tx(full_bar(s), bytes_all);
+            const uint32_t dA = sA + s * kPAStage;
+            const uint32_t dB = sB + s * kPBStage;
+            const int k = kb * kBK;
+            if (!j.a_mn) {
+              if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, k, a0);
+            } else {
+              if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, a0, k);
+              if (a0 + 64 < j.a_ext) tma_load_2d_pair(dA + kBox, j.mA, fb, a0 + 64, k);
+            }
+            if (!j.b_mn) {
+              if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, k, b0);
+            } else {
+              if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, b0, j.bk0 + k);
+              if (b0 + 64 < j.b_ext) tma_load_2d_pair(dB + kBox, j.mB, fb, b0 + 64, j.bk0 + k);
+            }
+            ++issued;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        long long u;
+        if constexpr (kDynamic) {
+          u = fetch_unit(k);
+        } else {
+          u = static_unit(k);
+        }
+        if (u < 0) break;
+        const Job j = make_job(P, u);
+        if (j.type < 0) break;
+        const uint32_t idesc = idesc_bf16_f32(kPairM, kBN, j.a_mn, j.b_mn);
+        const uint32_t a_lbo = j.a_mn ? 8192u : 16u, b_lbo = j.b_mn ? 8192u : 16u;
+        const uint32_t a_kstep = j.a_mn ? 2048u : 32u, b_kstep = j.b_mn ? 2048u : 32u;
+        for (int t = 0; ok && t < j.ntiles; ++t, ++tc) {
+          const int acc = tc & 1;
+          const uint32_t use = tc >> 1;
+          if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * kBN;
+          for (int kb = 0; kb < j.kbs; ++kb, ++it) {
+            const int s = it % kPStages;
+            const uint32_t ph = (it / kPStages) & 1u;
+            if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_s = sA + s * kPAStage, b_s = sB + s * kPBStage;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k) {
+              const uint64_t ad = smem_desc_sw128(a_s + k * a_kstep, a_lbo, 1024u);
+              const uint64_t bd = smem_desc_sw128(b_s + k * b_kstep, b_lbo, 1024u);
+              umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair_both(empty_bar(s));
+          }
+          if (ok) umma_commit_pair_both(tfull_bar(acc));
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const int row_off = kBM * static_cast<int>(rank) + row_in_tile;
+    const bool ep_leader = threadIdx.x == 64;
+    uint32_t tc = 0;
+    bool go = true;
+    for (uint32_t k = 0; go; ++k) {
+      long long u;
+      if constexpr (kDynamic) {
+        if (ep_leader) *ep_unit = static_cast<int>(fetch_unit(k));
+        epilogue_bar();
+        u = *ep_unit;
+      } else {
+        u = static_unit(k);
+      }
+      if (u < 0) break;
+      const Job j = make_job(P, u);
+      if (j.type < 0) break;
+      typename EpiFwd::State fst;
+      if constexpr (Mode == kModeFwd) EpiFwd::begin_unit(P.ep, fst, j.mt * kPairM + row_off, 0, 0);
+      for (int t = 0; t < j.ntiles; ++t, ++tc) {
+        const int acc = tc & 1;
+        const uint32_t use = tc >> 1;
+        if (ep_leader) {
+          bool ok = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, err);
+          if constexpr (Mode == kModeBwd) {
+            const BwdPlan& pl = P.plan;
+            if (ok && j.type == kUnitR && j.c >= kDxBuffers) {
+              const int c3 = j.c - kDxBuffers;
+              ok = wait_counter_bounded(P.bufdone + c3,
+                                        2u * static_cast<uint32_t>(bwd_nH(pl) + bwd_nD(pl, c3)),
+                                        abort_flag, err);
+            }
+            if (ok && j.type == kUnitH && j.c >= 1) {
+              ok = wait_counter_bounded(
+                  P.hdone + (static_cast<size_t>(j.c - 1) * pl.MT + j.mt) * pl.NH + j.nt, 2u,
+                  abort_flag, err);
+            }
+          }
+          *ep_ok = ok ? 1 : 0;
+        }
+        epilogue_bar();
+        if (!*ep_ok) {
+          go = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN;
+        const int row = j.mt * kPairM + row_off;
+        if constexpr (Mode == kModeFwd) {
+          EpiFwd::tile(P.ep, fst, taddr, j.nt + t);
+        } else if constexpr (Mode == kModeGemm) {
+          EpiStore::State st;
+          EpiStore::begin_unit(P.ep, st, row, 0, 0);
+          EpiStore::tile(P.ep, st, taddr, j.nt);
+        } else {
+          const BwdPlan& pl = P.plan;
+          if (j.type == kUnitR) {
+            EpiDlogits::Params p;
+            p.targets = P.targets;
+            p.lse = P.lse;
+            p.entropy = P.entropy;
+            p.dlogp = P.dlogp;
+            p.dentropy = P.dentropy;
+            p.dX = P.dx[j.c % kDxBuffers];
+            p.err = err;
+            p.T = pl.T;
+            p.V = pl.V;
+            p.c0 = j.c * pl.ldx;
+            p.ldx = pl.ldx;
+            p.scale_log2 = P.scale_log2;
+            p.inv_tau = P.inv_tau;
+            EpiDlogits::State st;
+            EpiDlogits::begin_unit(p, st, row, 0, 0);
+            EpiDlogits::tile(p, st, taddr, j.nt, &P.maps.dx_st[j.c % kDxBuffers],
+                             sStage + q * 4096u, lane, row - lane);
+          } else if (j.type == kUnitH) {
+            EpiDh::Params p;
+            p.acc = P.dh_acc;
+            p.out = P.dhidden;
+            p.T = pl.T;
+            p.H = pl.H;
+            p.mode = pl.NC == 1          ? EpiDh::kOnly
+                     : j.c == 0          ? EpiDh::kFirst
+                     : j.c == pl.NC - 1  ? EpiDh::kLast
+                                         : EpiDh::kMiddle;
+            EpiDh::State st;
+            EpiDh::begin_unit(p, st, row, 0, 0);
+            EpiDh::tile(p, st, taddr, j.nt);
+          } else {
+            EpiStore::Params p;
+            p.out = P.dW + static_cast<size_t>(j.c) * pl.ldx * pl.H;
+            p.rows = bwd_chunk_valid(pl, j.c);
+            p.ncols = pl.H;
+            p.ld = pl.H;
+            EpiStore::State st;
+            EpiStore::begin_unit(p, st, row, 0, 0);
+            EpiStore::tile(p, st, taddr, j.nt);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+        if constexpr (Mode == kModeBwd) {
+          if (j.type == kUnitR && lane == 0) bulk_wait_all();  // dX tiles written
+          epilogue_bar();  // every store of this CTA's half of the unit is done or issued
+          if (ep_leader) {
+            const BwdPlan& pl = P.plan;
+            fence_proxy_async_global();
+            __threadfence();
+            if (j.type == kUnitR) {
+              atomicAdd(P.rdone_m + static_cast<size_t>(j.c) * pl.MT + j.mt, 1u);
+              atomicAdd(P.rdone_j + static_cast<size_t>(j.c) * pl.RT_full + j.nt, 1u);
+            } else if (j.type == kUnitH) {
+              atomicAdd(P.hdone + (static_cast<size_t>(j.c) * pl.MT + j.mt) * pl.NH + j.nt, 1u);
+              atomicAdd(P.bufdone + j.c, 1u);
+            } else {
+              atomicAdd(P.bufdone + j.c, 1u);
+            }
+          }
+        }
+      }
+      if constexpr (Mode == kModeFwd) {
+        if (go) EpiFwd::end_unit(P.ep, fst, j.nt / P.group);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // Unwind after a timed-out wait: let TMA loads and MMAs in flight finish
+    // before the shared memory and TMEM they touch go away.
+    if (warp == 0 && lane == 0 && leader) {
+      const uint32_t first = issued > static_cast<uint32_t>(kPStages) ? issued - kPStages : 0u;
+      for (uint32_t i = first; i < issued; ++i)
+        mbar_wait_drain(full_bar(i % kPStages), (i / kPStages) & 1u);
+    }
+    if (warp == 1 && lane == 0 && leader) {
+      umma_commit_pair_both(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 2000000ull) __nanosleep(1000);  // 2 ms for the peer's copies
+    __syncthreads();
+  }
+  cluster_sync();  // neither CTA frees TMEM or exits while the other may still signal it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
+}
+
+}  // namespace rlk

@@ -68,10 +68,10 @@ int main(int argc, char** argv) {
     } else {
       const int vt = c == P.NC - 1 ? P.VT_last : P.VT_full;
       if (a >= vt || b >= P.NH) { printf("D range\n"); return 1; }
-      if ((long long)c * P.ldx + a * kBM >= V) { printf("D tile past V\n"); return 1; }
-      if (a * kBM + kBM > bwd_rt(P, c) * kBN) { printf("D reads unwritten dX columns\n"); return 1; }
+      if ((long long)c * P.ldx + a * kPairM >= V) { printf("D tile past V\n"); return 1; }
+      if (a * kPairM + kPairM > bwd_rt(P, c) * kBN) { printf("D reads unwritten dX columns\n"); return 1; }
       for (int m = 0; m < P.MT; ++m) {
-        const long long d = at(kUnitR, c, m, a / 2);
+        const long long d = at(kUnitR, c, m, a);
         if (d < 0 || d >= u) { printf("D dep on R not earlier\n"); return 1; }
       }
     }
