@@ -242,17 +242,23 @@ def run_ours(args):
         ms_max = float(t.item())
     flags = binding.rlk_read_device_error(ws)
 
-    # ---------------------------------------------------------------- forward kernel alone
-    fe0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    fe1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    for _ in range(3):
-        binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
-    for i in range(args.steps):
-        fe0[i].record(stream)
-        binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
-        fe1[i].record(stream)
-    torch.cuda.synchronize()
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(fe0, fe1))
+    # ---------------------------------------------------------------- each pass alone
+    def per_call_ms(fn, n):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    fwd_ms = per_call_ms(lambda: binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws,
+                                                             out=(logp, ent, lse)), args.steps)
+    bwd_ms = per_call_ms(lambda: binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent, dl, de,
+                                                             ws, out=(dH, dW)), args.steps)
 
     # ---------------------------------------------------------------- end to end, host buffers
     hid_h = torch.from_numpy(w.hidden.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -305,7 +311,8 @@ def run_ours(args):
     flops_tok = 8.0 * H * V
     step_tflops = flops_tok * T / (ms_max * 1e-3) / 1e12
     fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
-    launches_per_step = 3      # forward GEMM, combine, fused backward
+    bwd_tflops = 6.0 * T * H * V / (bwd_ms * 1e-3) / 1e12
+    launches_per_step = 3      # forward pair kernel, combine, backward pair kernel
     value = world * T / (ms_max * 1e-3)
     line = {
         "metric": METRIC,
@@ -326,12 +333,19 @@ def run_ours(args):
         "pct_of_bf16_peak": {"burst": step_tflops / pk["bf16_tflops"],
                              "sustained": step_tflops / pk["bf16_tflops_sustained"],
                              "datasheet_2250": step_tflops / 2250.0, "peaks": src},
-        "roofline": {"kernel": "forward: fused LM-head GEMM + online logsumexp/entropy "
-                               "+ target gather (+ combine), timed alone",
-                     "bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": fwd_tflops / pk["bf16_tflops"],
+        "roofline": {"kernel": "backward: one persistent pair-kernel launch (logits recompute + "
+                               "dlogits, dHidden and dW GEMMs), timed alone",
+                     "bound": "tensor", "achieved": bwd_tflops, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": bwd_tflops / pk["bf16_tflops"],
+                     "frac_of_sustained": bwd_tflops / pk["bf16_tflops_sustained"],
                      "traffic": None, "peak_source": src + " burst bf16",
-                     "flops_per_launch": 2.0 * T * H * V, "ms_per_launch": fwd_ms},
+                     "flops_per_launch": 6.0 * T * H * V, "ms_per_launch": bwd_ms},
+        "fwd_roofline": {"kernel": "forward: pair-kernel GEMM + online logsumexp/entropy + "
+                                   "target gather, with its combine, timed alone",
+                         "bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": fwd_tflops / pk["bf16_tflops"],
+                         "traffic": None, "peak_source": src + " burst bf16",
+                         "flops_per_launch": 2.0 * T * H * V, "ms_per_launch": fwd_ms},
         "step_roofline": {"bound": "tensor", "achieved": step_tflops,
                           "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                           "frac": step_tflops / pk["bf16_tflops_sustained"],

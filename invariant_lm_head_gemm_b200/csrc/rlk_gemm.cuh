@@ -1,31 +1,11 @@
-// rlk_gemm.cuh -- the one tensor-core mainloop behind every linear-logp
-// kernel, and the epilogues that turn its accumulator tiles into the
-// operator's results.
+// rlk_gemm.cuh -- tile constants, the epilogues that turn 128 x 256 fp32
+// accumulator tiles (one CTA's half of a pair tile, read from TMEM 32 columns
+// at a time) into the operator's results, and the forward's fixed-order
+// combine.  The mainloop that feeds them is pair_kernel (rlk_kernel.cuh).
 //
-// Mainloop.  D[M,N] = sum_k A[m,k] B[n,k] in 128 x 256 output tiles, bf16
-// operands, fp32 accumulation in tensor memory (TMEM).  Persistent CTAs (one
-// per SM, 192 threads, ~193 KB of shared memory) walk a static list of
-// "units"; a unit is one 128-row M tile and `group` consecutive 256-column N
-// tiles, processed in ascending order.  Warp roles:
-//   warp 0     TMA producer: 4-stage ring of (A 128x64, B 256x64) bf16 tiles,
-//              128-byte swizzled, one mbarrier pair per stage;
-//   warp 1     allocates 512 TMEM columns (two 256-column fp32 accumulators)
-//              and issues tcgen05.mma (M=128, N=256, K=16) from one thread;
-//   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane),
-//              reads it 32 columns at a time with tcgen05.ld and hands the
-//              values to the epilogue policy.
-// The accumulator is double buffered so the epilogue of tile i overlaps the
-// MMAs of tile i+1.  Every pipeline wait is bounded (rlk_ptx.cuh).
-//
-// Operands may be K-major (row of A / B contiguous along K) or MN-major
-// (contiguous along M / N); the instruction descriptor's transpose bits and
-// the shared-memory descriptors handle both, so the backward GEMMs read
-// dlogits, W and hidden in place without transposed copies.
-//
-// Batch invariance.  Each output element is produced by one CTA with a K
-// loop of fixed order and fixed instruction shape, and every epilogue works
-// row by row; nothing depends on how many rows the problem has or on which
-// CTA runs a unit.
+// Batch invariance.  Every epilogue works row by row in a fixed column order,
+// and each accumulator element comes from one fixed K loop; nothing depends on
+// how many rows the problem has or on which CTA pair runs a tile.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -38,39 +18,13 @@ constexpr int kBM = 128;     // accumulator rows per CTA
 constexpr int kPairM = 256;  // accumulator rows per CTA pair
 constexpr int kBN = 256;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
-constexpr uint32_t kAStage = kBM * kBK * 2;  // 16 KB
-constexpr uint32_t kBStage = kBN * kBK * 2;  // 32 KB
 constexpr uint32_t kBox = 64 * 64 * 2;       // one MN-major 64x64 box, 8 KB
-constexpr int kNumBars = 2 * kStages + 5;
-constexpr size_t kSmemBytes = 1024 + kStages * (kAStage + kBStage) + kNumBars * 8 + 16;
 
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 constexpr float kLn2 = 0.6931471805599453f;    // ln(2)
 constexpr float kMaskLogit = -1.0e30f;         // stands for -inf without producing NaN
-
-struct Sched {
-  int num_m_tiles;   // ceil(M / kBM)
-  int num_n_tiles;   // ceil(N / kBN)
-  int group;         // N tiles per unit
-  int num_groups;    // ceil(num_n_tiles / group)
-  int num_units;     // num_m_tiles * num_groups
-  int num_k_blocks;  // ceil(K / kBK)
-  int a_m_off, a_k_off;  // tensor-map coordinate offsets of A
-  int b_n_off, b_k_off;  // and of B
-  int a_mn_extent;   // extent of A's M coordinate in its tensor map
-  int b_mn_extent;   // extent of B's N coordinate in its tensor map
-};
-
-__device__ __forceinline__ void decode_unit(const Sched& sc, int u, int& mt, int& g, int& nt0,
-                                            int& nt1) {
-  mt = u % sc.num_m_tiles;
-  g = u / sc.num_m_tiles;
-  nt0 = g * sc.group;
-  nt1 = min(nt0 + sc.group, sc.num_n_tiles);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -80,7 +34,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // =====================================================================
 // Epilogue policies.  Each provides Params, State and
 //   begin_unit(p, st, row, mt, g)   once per unit, row = global M index
-//   tile(p, st, taddr, nt)          once per 128x256 accumulator tile
+//   tile(p, st, taddr, nt, ...)     once per 128x256 accumulator tile
 //   end_unit(p, st, g)              once per unit
 // =====================================================================
 
@@ -383,211 +337,6 @@ struct EpiStore {
 
   __device__ static void end_unit(const Params&, State&, int) {}
 };
-
-// =====================================================================
-// The persistent kernel.
-// =====================================================================
-template <class Epi, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const Sched sc, const typename Epi::Params ep, uint32_t* err) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  const uint32_t sA = smem_u32(smem);
-  const uint32_t sB = sA + kStages * kAStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * (kAStage + kBStage));
-  const uint32_t bar0 = smem_u32(bars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
-  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
-    }
-    mbar_init(drain_bar, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  uint32_t issued = 0;  // producer: k-blocks whose loads were issued
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < sc.num_units; u += gridDim.x) {
-        int mt, g, nt0, nt1;
-        decode_unit(sc, u, mt, g, nt0, nt1);
-        for (int nt = nt0; ok && nt < nt1; ++nt) {
-          for (int kb = 0; kb < sc.num_k_blocks; ++kb) {
-            const int s = issued % kStages;
-            const uint32_t ph = (issued / kStages) & 1u;
-            if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
-              ok = false;
-              break;
-            }
-            const uint32_t dA = sA + s * kAStage;
-            const uint32_t dB = sB + s * kBStage;
-            const int ka = sc.a_k_off + kb * kBK;
-            const int kbb = sc.b_k_off + kb * kBK;
-            const int m0 = sc.a_m_off + mt * kBM;
-            const int n0 = sc.b_n_off + nt * kBN;
-            uint32_t bytes = 0;
-            if (!A_MN) {
-              bytes += kAStage;
-            } else {
-#pragma unroll
-              for (int j = 0; j < kBM / 64; ++j)
-                if (m0 + 64 * j < sc.a_mn_extent) bytes += kBox;
-            }
-            if (!B_MN) {
-              bytes += kBStage;
-            } else {
-#pragma unroll
-              for (int j = 0; j < kBN / 64; ++j)
-                if (n0 + 64 * j < sc.b_mn_extent) bytes += kBox;
-            }
-            mbar_arrive_expect_tx(full_bar(s), bytes);
-            if (!A_MN) {
-              tma_load_2d(dA, &tmA, full_bar(s), ka, m0);
-            } else {
-#pragma unroll
-              for (int j = 0; j < kBM / 64; ++j)
-                if (m0 + 64 * j < sc.a_mn_extent)
-                  tma_load_2d(dA + j * kBox, &tmA, full_bar(s), m0 + 64 * j, ka);
-            }
-            if (!B_MN) {
-              tma_load_2d(dB, &tmB, full_bar(s), kbb, n0);
-            } else {
-#pragma unroll
-              for (int j = 0; j < kBN / 64; ++j)
-                if (n0 + 64 * j < sc.b_mn_extent)
-                  tma_load_2d(dB + j * kBox, &tmB, full_bar(s), n0 + 64 * j, kbb);
-            }
-            ++issued;
-          }
-        }
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, A_MN, B_MN);
-      constexpr uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
-      constexpr uint32_t a_kstep = A_MN ? 2048u : 32u, b_kstep = B_MN ? 2048u : 32u;
-      uint32_t it = 0, tc = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < sc.num_units; u += gridDim.x) {
-        int mt, g, nt0, nt1;
-        decode_unit(sc, u, mt, g, nt0, nt1);
-        for (int nt = nt0; ok && nt < nt1; ++nt, ++tc) {
-          const int acc = tc & 1;
-          const uint32_t use = tc >> 1;
-          if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + acc * kBN;
-          for (int kb = 0; kb < sc.num_k_blocks; ++kb, ++it) {
-            const int s = it % kStages;
-            const uint32_t ph = (it / kStages) & 1u;
-            if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t a0 = sA + s * kAStage, b0 = sB + s * kBStage;
-#pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t ad = smem_desc_sw128(a0 + k * a_kstep, a_lbo, 1024u);
-              const uint64_t bd = smem_desc_sw128(b0 + k * b_kstep, b_lbo, 1024u);
-              umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
-            }
-            umma_commit(empty_bar(s));
-          }
-          if (ok) umma_commit(tfull_bar(acc));
-        }
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row_in_tile = q * 32 + lane;
-    uint32_t tc = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < sc.num_units; u += gridDim.x) {
-      int mt, g, nt0, nt1;
-      decode_unit(sc, u, mt, g, nt0, nt1);
-      typename Epi::State st;
-      Epi::begin_unit(ep, st, mt * kBM + row_in_tile, mt, g);
-      for (int nt = nt0; nt < nt1; ++nt, ++tc) {
-        const int acc = tc & 1;
-        const uint32_t use = tc >> 1;
-        int w = 1;
-        if (lane == 0) w = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, err) ? 1 : 0;
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * kBN;
-        Epi::tile(ep, st, taddr, nt);
-        tc_fence_before();
-        mbar_arrive(tempty_bar(acc));
-      }
-      if (ok) Epi::end_unit(ep, st, g);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (*abort_flag) {
-    // Unwind after a timed-out wait: let every TMA load still in flight land
-    // and every issued MMA finish before the memory they touch goes away.
-    if (warp == 0 && lane == 0) {
-      const uint32_t first = issued > static_cast<uint32_t>(kStages) ? issued - kStages : 0u;
-      for (uint32_t i = first; i < issued; ++i)
-        mbar_wait_drain(full_bar(i % kStages), (i / kStages) & 1u);
-    }
-    if (warp == 1 && lane == 0) {
-      umma_commit(drain_bar);
-      mbar_wait_drain(drain_bar, 0);
-    }
-    __syncthreads();
-  }
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
-}
 
 // Fixed-order merge of the forward's per-split triples, one thread per row:
 // lse = ln2 (M + log2 S), entropy = ln2 (log2 S - B / S),
