@@ -348,8 +348,10 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   P.inv_tau = 1.0f / temperature;
 
   if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
-  // Units wait on units of other CTAs, so every CTA must be resident.
-  if ((s = launch_pair<kModeBwd>(P, pl.total, true, st)) != RLK_OK) return s;
+  // Units wait on units claimed earlier, and only running CTA pairs claim
+  // units, so no pair ever waits on one that has not started: the launch needs
+  // no co-residency guarantee.
+  if ((s = launch_pair<kModeBwd>(P, pl.total, false, st)) != RLK_OK) return s;
   g_calls[1].fetch_add(1);
   return RLK_OK;
 }

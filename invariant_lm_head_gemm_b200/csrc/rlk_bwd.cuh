@@ -16,10 +16,11 @@
 //   H(c, m, n) needs H(c - 1, m, n)               (flag hdone[c - 1][m][n])
 //   R(c, ., .) overwrites buffer c % 3 only after every H(c - 3), D(c - 3)
 //                                                 (counter bufdone[c - 3])
-// CTA pair p runs units p, p + pairs, p + 2 pairs, ... in ascending order and
-// a unit only ever waits for smaller units, so with all CTAs resident (the
-// launch is cooperative) every wait ends; each wait is also time-bounded.
-// Both CTAs of a pair signal each unit, so the counters count CTA halves.
+// CTA pairs claim units from a global counter in ascending order and a unit
+// only ever waits for smaller units, all of them claimed earlier by pairs that
+// are running; so every wait ends without any co-residency guarantee (each
+// wait is also time-bounded).  Both CTAs of a pair signal each unit, so the
+// counters count CTA halves.
 // Producers of a counter store with generic stores, sync the epilogue warps,
 // then one thread fences and increments; consumers acquire, and fence the
 // async proxy before TMA reads of the data.
