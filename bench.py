@@ -138,6 +138,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def aggregate(ms_local, tokens_local):
+    """Across ranks: the slowest rank's step time and the tokens all ranks
+    processed (weak scaling: value = tokens / max time)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms_local), float(tokens_local)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+    n = torch.tensor([tokens_local], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(n.item())
+
+
 def rl_inputs(rank):
     from invariant_lm_head_gemm_b200 import workloads as wl
     w = wl.rl_step(3 + 1000 * rank, with_weight=False)
@@ -264,11 +279,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max, tokens_all = aggregate(ms, T)
     flags = binding.rlk_read_device_error(ws)
 
     # ---------------------------------------------------------------- each pass alone
@@ -318,11 +329,7 @@ def run_ours(args):
     ee1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = ee0.elapsed_time(ee1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms, _ = aggregate(ee0.elapsed_time(ee1) / args.steps, T)
     h2d = T * H * 2 + T * 8 + T * 4 + T * 4
     d2h = 2 * T * 4
 
@@ -339,11 +346,11 @@ def run_ours(args):
     pk, src = peaks()
     fwd_traffic, bwd_traffic = measured_traffic()
     flops_tok = 8.0 * H * V
-    step_tflops = flops_tok * T / (ms_max * 1e-3) / 1e12
+    step_tflops = flops_tok * tokens_all / world / (ms_max * 1e-3) / 1e12
     fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = 6.0 * T * H * V / (bwd_ms * 1e-3) / 1e12
     launches_per_step = 3      # forward pair kernel, combine, backward pair kernel
-    value = world * T / (ms_max * 1e-3)
+    value = tokens_all / (ms_max * 1e-3)
     line = {
         "metric": METRIC,
         "value": value,
@@ -381,7 +388,7 @@ def run_ours(args):
                           "frac": step_tflops / pk["bf16_tflops_sustained"],
                           "flops_per_token": flops_tok, "peak_source": src + " sustained bf16"},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
