@@ -136,8 +136,27 @@ __host__ inline long long bwd_total_units(const BwdPlan& P) {
 __host__ __device__ inline BwdUnit bwd_seg_R(const BwdPlan& P, int c, long long i) {
   return BwdUnit{kUnitR, c, static_cast<int>(i % P.MT), static_cast<int>(i / P.MT)};
 }
+// dHidden units of one chunk in groups of kHGroup row blocks: inside a group
+// the row block varies fastest, then the column block.  The units in flight
+// then share a few W column blocks and a few dX row blocks, so neither the
+// chunk's W columns nor its dX rows have to stream from DRAM many times.
+constexpr int kHGroup = 8;
+
 __host__ __device__ inline BwdUnit bwd_seg_H(const BwdPlan& P, int c, long long i) {
-  return BwdUnit{kUnitH, c, static_cast<int>(i / P.NH), static_cast<int>(i % P.NH)};
+  const long long full = P.MT / kHGroup;
+  const long long per_group = static_cast<long long>(kHGroup) * P.NH;
+  int m, n;
+  if (i < full * per_group) {
+    const long long g = i / per_group, r = i % per_group;
+    n = static_cast<int>(r / kHGroup);
+    m = static_cast<int>(g * kHGroup + r % kHGroup);
+  } else {
+    const int rem = P.MT % kHGroup;
+    const long long r = i - full * per_group;
+    n = static_cast<int>(r / rem);
+    m = static_cast<int>(full * kHGroup + r % rem);
+  }
+  return BwdUnit{kUnitH, c, m, n};
 }
 __host__ __device__ inline BwdUnit bwd_seg_D(const BwdPlan& P, int c, long long i) {
   return BwdUnit{kUnitD, c, static_cast<int>(i / P.NH), static_cast<int>(i % P.NH)};
