@@ -256,9 +256,23 @@ def run_ours(args):
     dW = torch.empty(V, H, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # N > 1: the data-parallel exchange of dW (deterministic reduce-scatter:
+    # one NCCL all-to-all of vocab slices, then the rank-ordered sum)
+    use_rs = world > 1 and not args.no_dw_reduce
+    if use_rs:
+        from invariant_lm_head_gemm_b200 import dp
+        per = -(-V // world)
+        rs_recv = torch.empty(world, per, H, dtype=torch.float32, device=dev)
+        rs_out = torch.empty(per, H, dtype=torch.float32, device=dev)
+
+    def exchange():
+        if use_rs:
+            dp.reduce_scatter_dw(dW, rs_recv, rs_out)
+
     def step():
         binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
         binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent, dl, de, ws, out=(dH, dW))
+        exchange()
 
     def barrier():
         if world > 1:
@@ -315,6 +329,7 @@ def run_ours(args):
         de.copy_(de_h, non_blocking=True)
         binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(res[0], res[1], lse))
         binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, res[1], dl, de, ws, out=(dH, dW))
+        exchange()
         out_h.copy_(res, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -349,7 +364,8 @@ def run_ours(args):
     step_tflops = flops_tok * tokens_all / world / (ms_max * 1e-3) / 1e12
     fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = 6.0 * T * H * V / (bwd_ms * 1e-3) / 1e12
-    launches_per_step = 3      # forward pair kernel, combine, backward pair kernel
+    launches_per_step = 3 + (1 if use_rs else 0)   # fwd pair kernel, combine, bwd pair
+                                                    # kernel (+ the ordered sum of dW)
     value = tokens_all / (ms_max * 1e-3)
     line = {
         "metric": METRIC,
@@ -391,6 +407,11 @@ def run_ours(args):
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
+        "dw_exchange": {"included": bool(use_rs),
+                        "kind": "deterministic reduce-scatter of dW: NCCL all-to-all of "
+                                "vocab-row slices, then the rank-ordered sum (rlk_sum_ordered)",
+                        "bytes_sent_per_rank": (int((world - 1) * -(-V // world) * H * 4)
+                                                if use_rs else 0)},
         "clocks": clk.summary(),
         "device_error_flags": flags,
     }
@@ -438,6 +459,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=48)
     ap.add_argument("--ref-rows", type=int, default=2)
+    ap.add_argument("--no-dw-reduce", action="store_true",
+                    help="N > 1: leave out the deterministic dW reduce-scatter from the step")
     ap.add_argument("--profile", choices=["fwd", "bwd"], default=None,
                     help="run a small case for an ncu capture instead of the benchmark")
     ap.add_argument("--T", type=int, default=2048, help="rows of the --profile case")

@@ -136,16 +136,31 @@ rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W
                                        float temperature, float* logp, float* entropy,
                                        float* lse, void* stream);
 
-/* Self-check of the tensor-core mainloop shared by every kernel above:
- * C[M,N] fp32 = sum_k A[m,k] B[n,k] with bf16 inputs and fp32 accumulation.
- * a_mn_major == 0: A is stored [M,K] (K contiguous); != 0: stored [K,M].
- * b_mn_major == 0: B is stored [N,K]; != 0: stored [K,N].  M, N, K >= 1 and
- * multiples of 8.  Not part of the operator; the pages have no counterpart.
- * Needs a workspace of rlk_gemm_workspace_bytes() bytes for its error word. */
+/* Batch-invariant deterministic dense GEMM on the same tensor-core mainloop as
+ * every kernel above (also its self-check): C[M,N] fp32 = sum_k A[m,k] B[n,k]
+ * with bf16 inputs and fp32 accumulation, each row of C bitwise independent of
+ * the other rows of A and repeatable.  The pages run such a route for the
+ * dense FFN and LoRA linear ("rlkernel.ffn.qwen3.deterministic.v1",
+ * h100-cp-gradient.json runtime readbacks; lora_gate, h3-runtime-integration-
+ * b200 report).  a_mn_major == 0: A is stored [M,K] (K contiguous); != 0:
+ * stored [K,M].  b_mn_major == 0: B is stored [N,K]; != 0: stored [K,N].
+ * M, N, K >= 1; K and N multiples of 8, and M too when a_mn_major.  Needs a
+ * workspace of rlk_gemm_workspace_bytes() bytes for its error word. */
 size_t rlk_gemm_workspace_bytes(void);
 rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, int64_t N,
                              int64_t K, int a_mn_major, int b_mn_major, float* C,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Fixed-order sum out[i] = ((parts[0][i] + parts[1][i]) + parts[2][i]) + ...
+ * over nparts (1..64) equally sized fp32 device buffers of `count` elements;
+ * `parts` is a HOST array of device pointers.  The data-parallel exchange of
+ * dW uses it: every rank's partial dW slice reaches the slice's owner, which
+ * adds them in rank order, so the result is bitwise the same whatever order
+ * the slices arrive in.  (The pages' deterministic TP collectives stage
+ * through CUDA-IPC buffers: VIME Qwen3-8B TP4/CP2 page, "Required gates".)
+ * out may alias parts[0].  Enqueued on `stream`; no allocation. */
+rlk_status rlk_sum_ordered(const float* const* parts, int nparts, float* out, int64_t count,
+                           void* stream);
 
 /* Provenance readback, in the spirit of the pages' per-module runtime
  * readbacks (h100-cp-gradient.json, runs[].validation.runtime_readbacks:

@@ -236,3 +236,26 @@ def rlk_linear_logp_fwd_noalloc(hidden, W, targets, temperature, out=None, strea
                        _ptr(logp), _ptr(entropy), _ptr(lse), _stream(stream)),
            "rlk_linear_logp_fwd_noalloc")
     return logp, entropy, lse
+
+
+_sum_fn = None
+
+
+def rlk_sum_ordered(parts, out=None, stream=None):
+    """out = ((parts[0] + parts[1]) + parts[2]) + ... elementwise in fp32, in
+    list order (1..64 equally shaped contiguous CUDA fp32 tensors)."""
+    global _sum_fn
+    if _sum_fn is None:
+        f = lib().rlk_sum_ordered
+        f.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, _P, _I64, _P]
+        f.restype = ctypes.c_int
+        _sum_fn = f
+    n = parts[0].numel()
+    for t in parts:
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or t.numel() != n:
+            raise ValueError("parts must be contiguous CUDA fp32 tensors of equal size")
+    if out is None:
+        out = torch.empty_like(parts[0])
+    arr = (ctypes.c_void_p * len(parts))(*[t.data_ptr() for t in parts])
+    _check(_sum_fn(arr, len(parts), _ptr(out), n, _stream(stream)), "rlk_sum_ordered")
+    return out

@@ -230,6 +230,7 @@ rlk_status enqueue_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   a.ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
   a.ep.T = static_cast<int>(T);
   a.ep.V = static_cast<int>(V);
+  a.ep.G = static_cast<int>(fwd_groups(V));
   a.ep.scale_log2 = kLog2e / temperature;
   a.err = err;
   a.MT = static_cast<int>(ceil_div(T, kPairM));
@@ -240,7 +241,7 @@ rlk_status enqueue_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   a.total = static_cast<long long>(a.MT) * a.NG;
   rlk_status s = launch_pair<kModeFwd>(a, a.total, false, st);
   if (s != RLK_OK) return s;
-  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 256)), 256, 0, st>>>(
+  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 8)), 256, 0, st>>>(
       a.ep.part_m, a.ep.part_s, a.ep.part_b, a.ep.ytgt, targets, static_cast<int>(T),
       static_cast<int>(V), a.NG, logp, entropy, lse, err);
   return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
@@ -362,8 +363,9 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
                              int64_t K, int a_mn_major, int b_mn_major, float* C,
                              void* workspace, size_t workspace_bytes, void* stream) {
   if (M <= 0 || N <= 0 || K <= 0) return RLK_ERR_INVALID_ARG;
-  if (M % 8 || N % 8 || K % 8 || M >= (int64_t{1} << 31) || N >= (int64_t{1} << 31) ||
-      K >= (int64_t{1} << 31))
+  // 16-byte row pitches for every tensor map and for C's vector stores
+  if (K % 8 || N % 8 || (a_mn_major && M % 8) || M >= (int64_t{1} << 31) ||
+      N >= (int64_t{1} << 31) || K >= (int64_t{1} << 31))
     return RLK_ERR_UNSUPPORTED_SHAPE;
   if (!A || !B || !C || !workspace) return RLK_ERR_INVALID_ARG;
   if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(workspace, 256))
@@ -433,6 +435,78 @@ const char* rlk_status_string(rlk_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fixed-order sum of equally shaped fp32 buffers (the data-parallel exchange
+// of dW: every rank's partial slice arrives at the slice's owner, which adds
+// them in rank order, so the sum never depends on arrival order).
+// ---------------------------------------------------------------------------
+namespace rlk {
+namespace {
+
+constexpr int kMaxSumParts = 64;
+
+struct SumParts {
+  const float* p[kMaxSumParts];
+};
+
+__global__ void __launch_bounds__(256) sum_ordered_vec4_kernel(const __grid_constant__ SumParts P,
+                                                               int n, float4* out,
+                                                               int64_t count4) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(P.p[0])[i];
+    for (int k = 1; k < n; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(P.p[k])[i];
+      acc.x = acc.x + v.x;
+      acc.y = acc.y + v.y;
+      acc.z = acc.z + v.z;
+      acc.w = acc.w + v.w;
+    }
+    out[i] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(256) sum_ordered_kernel(const __grid_constant__ SumParts P, int n,
+                                                          float* out, int64_t count) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float acc = P.p[0][i];
+    for (int k = 1; k < n; ++k) acc = acc + P.p[k][i];
+    out[i] = acc;
+  }
+}
+
+}  // namespace
+}  // namespace rlk
+
+extern "C" rlk_status rlk_sum_ordered(const float* const* parts, int nparts, float* out,
+                                      int64_t count, void* stream) {
+  if (!parts || !out || nparts < 1 || nparts > kMaxSumParts || count < 0)
+    return RLK_ERR_INVALID_ARG;
+  if (count == 0) return RLK_OK;
+  SumParts P;
+  bool vec = aligned(out, 16) && count % 4 == 0;
+  for (int k = 0; k < nparts; ++k) {
+    if (!parts[k]) return RLK_ERR_INVALID_ARG;
+    if (!aligned(parts[k], 4)) return RLK_ERR_MISALIGNED;
+    vec = vec && aligned(parts[k], 16);
+    P.p[k] = parts[k];
+  }
+  if (!aligned(out, 4)) return RLK_ERR_MISALIGNED;
+  int sms = 0;
+  rlk_status s = check_device(&sms);
+  if (s != RLK_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t items = vec ? count / 4 : count;
+  const unsigned blocks =
+      static_cast<unsigned>(std::min<int64_t>(ceil_div(items, 256), static_cast<int64_t>(sms) * 8));
+  if (vec)
+    sum_ordered_vec4_kernel<<<blocks, 256, 0, st>>>(P, nparts, reinterpret_cast<float4*>(out), items);
+  else
+    sum_ordered_kernel<<<blocks, 256, 0, st>>>(P, nparts, out, items);
+  return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------------------
 // Forward without a caller-provided workspace.

@@ -46,12 +46,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 struct EpiFwd {
   struct Params {
     const int64_t* targets;
-    float* part_m;
+    float* part_m;  // [T][G] (row-major: a row's splits are contiguous)
     float* part_s;
     float* part_b;
     float* ytgt;
     int T;
     int V;
+    int G;             // vocab splits
     float scale_log2;  // log2(e) / tau
   };
   struct State {
@@ -111,7 +112,7 @@ struct EpiFwd {
 
   __device__ static void end_unit(const Params& p, State& st, int g) {
     if (st.valid) {
-      const size_t i = static_cast<size_t>(g) * p.T + st.row;
+      const size_t i = static_cast<size_t>(st.row) * p.G + g;
       p.part_m[i] = st.m;
       p.part_s[i] = st.s;
       p.part_b[i] = st.b;
@@ -338,9 +339,27 @@ struct EpiStore {
   __device__ static void end_unit(const Params&, State&, int) {}
 };
 
-// Fixed-order merge of the forward's per-split triples, one thread per row:
+// Fixed-order merge of the forward's per-split triples into
 // lse = ln2 (M + log2 S), entropy = ln2 (log2 S - B / S),
 // logp = ln2 (y_target - M - log2 S).
+// One warp per row: lane l merges splits l, l + 32, l + 64, ... in ascending
+// order, then the lanes combine by an xor butterfly.  merge(a, b) and
+// merge(b, a) are bitwise equal (max and + are commutative), so every lane
+// ends with the same triple, and the order depends only on the split count.
+struct Triple {
+  float m, s, b;
+};
+
+__device__ __forceinline__ Triple merge_triple(Triple x, Triple y) {
+  const float mn = fmaxf(x.m, y.m);
+  const float ax = ex2_approx(x.m - mn), ay = ex2_approx(y.m - mn);
+  Triple r;
+  r.m = mn;
+  r.s = ax * x.s + ay * y.s;
+  r.b = ax * fmaf(x.m - mn, x.s, x.b) + ay * fmaf(y.m - mn, y.s, y.b);
+  return r;
+}
+
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ pm,
                                                       const float* __restrict__ ps,
                                                       const float* __restrict__ pb,
@@ -349,28 +368,30 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
                                                       int V, int G, float* __restrict__ logp,
                                                       float* __restrict__ entropy,
                                                       float* __restrict__ lse, uint32_t* err) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= T) return;
-  float M = kMaskLogit, S = 0.f, B = 0.f;
-  for (int g = 0; g < G; ++g) {
-    const size_t i = static_cast<size_t>(g) * T + t;
-    const float m = pm[i], s = ps[i], b = pb[i];
-    const float mn = fmaxf(M, m);
-    const float a1 = ex2_approx(M - mn);
-    const float a2 = ex2_approx(m - mn);
-    B = a1 * fmaf(M - mn, S, B) + a2 * fmaf(m - mn, s, b);
-    S = a1 * S + a2 * s;
-    M = mn;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;  // warp-uniform
+  const size_t base = static_cast<size_t>(t) * G;
+  Triple acc{kMaskLogit, 0.f, 0.f};
+  for (int g = lane; g < G; g += 32) acc = merge_triple(acc, Triple{pm[base + g], ps[base + g], pb[base + g]});
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    Triple o;
+    o.m = __shfl_xor_sync(0xffffffffu, acc.m, off);
+    o.s = __shfl_xor_sync(0xffffffffu, acc.s, off);
+    o.b = __shfl_xor_sync(0xffffffffu, acc.b, off);
+    acc = merge_triple(acc, o);
   }
-  const float l2s = log2f(S);
-  lse[t] = kLn2 * (M + l2s);
-  entropy[t] = kLn2 * (l2s - B / S);
+  if (lane != 0) return;
+  const float l2s = log2f(acc.s);
+  lse[t] = kLn2 * (acc.m + l2s);
+  entropy[t] = kLn2 * (l2s - acc.b / acc.s);
   const int64_t tg = targets[t];
   if (tg < 0 || tg >= V) {
     logp[t] = __int_as_float(0x7fc00000);
     atomicOr(err, kDevErrTarget);
   } else {
-    logp[t] = kLn2 * ((ytgt[t] - M) - l2s);
+    logp[t] = kLn2 * ((ytgt[t] - acc.m) - l2s);
   }
 }
 

@@ -105,7 +105,9 @@ def test_backward_argument_errors(L):
 def test_gemm_argument_errors(L):
     g = L.rlk_gemm_bf16_f32
     assert g(A16, A16, 0, 8, 8, 0, 0, A16, A256, 256, None) == INVALID
-    assert g(A16, A16, 12, 8, 8, 0, 0, A16, A256, 256, None) == SHAPE
+    assert g(A16, A16, 12, 8, 8, 1, 0, A16, A256, 256, None) == SHAPE    # MN-major A: M % 8
+    assert g(A16, A16, 8, 12, 8, 0, 0, A16, A256, 256, None) == SHAPE    # N % 8
+    assert g(A16, A16, 8, 8, 12, 0, 0, A16, A256, 256, None) == SHAPE    # K % 8
     assert g(None, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == INVALID
     assert g(A16 + 2, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == MISALIGNED
     assert g(A16, A16, 8, 8, 8, 0, 0, A16, A256, 255, None) == WS_SMALL

@@ -55,3 +55,50 @@ def test_single_process_aggregate_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.aggregate(12.5, 5980) == (12.5, 5980.0)
+
+
+def _dw(rank, V, H):
+    import torch
+    g = torch.Generator().manual_seed(1000 + rank)
+    return torch.randn(V, H, generator=g)
+
+
+def _cpu_ordered_sum(parts, out):
+    acc = parts[0].clone()
+    for p in parts[1:]:
+        acc = acc + p
+    out.copy_(acc)
+
+
+def _rs_worker(rank, world, port, V, H, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from invariant_lm_head_gemm_b200 import dp
+    res, r0, r1 = dp.reduce_scatter_dw(_dw(rank, V, H), sum_fn=_cpu_ordered_sum)
+    out[rank] = (r0, r1, res.numpy().tobytes())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,V", [(2, 37), (3, 8), (2, 1)])
+def test_dw_reduce_scatter_is_the_rank_ordered_sum(world, V):
+    H = 8
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rs_worker, args=(world, _free_port(), V, H, out), nprocs=world, join=True)
+        res = dict(out)
+    full = _dw(0, V, H)
+    for r in range(1, world):
+        full = full + _dw(r, V, H)          # rank order
+    covered = 0
+    for r in range(world):
+        r0, r1, raw = res[r]
+        got = np.frombuffer(raw, dtype=np.float32).reshape(-1, H)[: r1 - r0]
+        assert np.array_equal(got.view(np.uint32), full[r0:r1].numpy().view(np.uint32))
+        covered += r1 - r0
+    assert covered == V
