@@ -136,6 +136,94 @@ rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W
                                        float temperature, float* logp, float* entropy,
                                        float* lse, void* stream);
 
+/* Vocab-parallel (tensor-parallel) forward, invariant to the TP degree.  The
+ * pages train the same model under TP2/CP4 and TP4/CP2 layouts and find the
+ * weights, gradient norms and tokens bitwise equal across the two runs
+ * (h100-cp-gradient.json, all_parameter_hash_comparisons[].bitwise_equal,
+ * gradient_norm_comparisons[].exactly_equal, tokens_equal).  Here each rank
+ * holds a contiguous shard of W whose first row v0 is a multiple of
+ * rlk_fwd_split_width() (512): the forward's vocab splits then fall wholly in
+ * one shard and every shard computes exactly the single-GPU split triples, so
+ * merging the gathered splits in global order gives logp / entropy / lse bit
+ * for bit equal to rlk_linear_logp_fwd, for any number of shards.
+ *
+ * rlk_linear_logp_fwd_shard: hidden [T,H] bf16, W_shard [V_shard,H] bf16 =
+ * rows v0 .. v0+V_shard-1 of the full [V,H] head, targets [T] (global vocab
+ * indices).  Writes the first ceil(V_shard / 512) columns of part_m, part_s,
+ * part_b, each [T][Gs] fp32 (row stride Gs, with ceil(V_shard / 512) <= Gs <=
+ * ceil(V / 512); give every shard the same Gs so that the buffers concatenate
+ * into the combine's layout), and ytgt[t] for the rows whose target lies in
+ * the shard (other rows of ytgt are left untouched).  The workspace holds only
+ * the device error word (256 bytes).  v0 not a multiple of 512, or V_shard
+ * not one either for a shard that does not end at V, gives
+ * RLK_ERR_UNSUPPORTED_SHAPE; a shard outside [0, V) or Gs out of range gives
+ * RLK_ERR_INVALID_ARG.
+ *
+ * rlk_linear_logp_combine: part_* laid out [nshards][T][Gs] (the shards' part_
+ * buffers one after another, as an all-gather delivers them), the last shard's
+ * unused columns ignored, (nshards-1)*Gs < ceil(V/512) <= nshards*Gs; ytgt [T] holds every row's target logit (each row's from the
+ * shard that owns its target).  Writes logp, entropy, lse [T] as
+ * rlk_linear_logp_fwd does; out-of-range targets give NaN logp and set
+ * RLK_DEVERR_TARGET in the workspace. */
+int64_t rlk_fwd_split_width(void);
+rlk_status rlk_linear_logp_fwd_shard(const rlk_bf16* hidden, const rlk_bf16* W_shard,
+                                     const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                     int64_t v0, int64_t V_shard, float temperature,
+                                     float* part_m, float* part_s, float* part_b, int64_t Gs,
+                                     float* ytgt, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+rlk_status rlk_linear_logp_combine(const float* part_m, const float* part_s, const float* part_b,
+                                   int64_t nshards, int64_t Gs, const float* ytgt,
+                                   const int64_t* targets, int64_t T, int64_t V, float* logp,
+                                   float* entropy, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* Vocab-parallel backward, invariant to the TP degree (same pages and fields
+ * as the vocab-parallel forward above).  The single-GPU backward adds the
+ * dHidden products of its vocab chunks (rlk_bwd_chunk_width(V) rows each, the
+ * last one ragged) in ascending chunk order in fp32 and rounds the sum to
+ * bf16 once.  A shard whose first row v0 is a multiple of the chunk width, and
+ * whose length is too unless it ends at V, holds whole chunks of the full
+ * head; it writes each chunk's fp32 product on its own, and
+ * rlk_dhidden_combine adds the products of all shards in global chunk order
+ * with the same additions and rounding.  dHidden and dW therefore equal
+ * rlk_linear_logp_bwd's bit for bit for any number of shards.
+ *
+ * rlk_bwd_chunk_width: vocab rows per backward chunk for a V-row head
+ * (min(8192, V rounded up to 256)); 0 for V outside [1, 2^31).
+ *
+ * rlk_linear_logp_bwd_shard: hidden, targets (global indices), lse, entropy,
+ * dlogp, dentropy as for rlk_linear_logp_bwd (lse, entropy of the full
+ * vocabulary, e.g. from rlk_linear_logp_combine); W_shard [V_shard,H] bf16 =
+ * rows v0 .. v0+V_shard-1 of the head.  Writes dW_shard [V_shard,H] fp32 (the
+ * shard's rows of dW) and the shard's chunk products into dh_parts, fp32 laid
+ * out [S][part_chunks][part_rows][H] with S = ceil(T / part_rows): the product
+ * of local chunk k for row t sits at slice t / part_rows, slot k, row
+ * t % part_rows (slots past the shard's chunks and rows past T are not
+ * written).  part_rows = T gives plain [chunk][T][H]; part_rows =
+ * ceil(T / ranks) puts each rank's row slice in one contiguous block, ready for
+ * an all-to-all.  part_chunks in [ceil(V_shard / width), ceil(V / width)].
+ * Workspace: rlk_linear_logp_workspace_bytes(T, H, V, 1) bytes (full V),
+ * 256-byte aligned.  Errors: v0 or V_shard off the chunk grid
+ * RLK_ERR_UNSUPPORTED_SHAPE; shard outside [0, V), part_rows < 1 or
+ * part_chunks out of range RLK_ERR_INVALID_ARG; otherwise as
+ * rlk_linear_logp_bwd.  T = 0 zeroes dW_shard.
+ *
+ * rlk_dhidden_combine: dh_parts [nparts][count] fp32 (16-byte aligned), the
+ * chunk products in global chunk order; writes out[i] = bf16 of
+ * ((p_0[i] + p_1[i]) + ...) + p_{nparts-1}[i], out [count] bf16 (8-byte
+ * aligned).  count must be a multiple of 4 (RLK_ERR_UNSUPPORTED_SHAPE). */
+int64_t rlk_bwd_chunk_width(int64_t V);
+rlk_status rlk_linear_logp_bwd_shard(const rlk_bf16* hidden, const rlk_bf16* W_shard,
+                                     const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                     int64_t v0, int64_t V_shard, float temperature,
+                                     const float* lse, const float* entropy, const float* dlogp,
+                                     const float* dentropy, float* dh_parts, int64_t part_rows,
+                                     int64_t part_chunks, float* dW_shard, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+rlk_status rlk_dhidden_combine(const float* dh_parts, int64_t nparts, int64_t count,
+                               rlk_bf16* out, void* stream);
+
 /* Batch-invariant deterministic dense GEMM on the same tensor-core mainloop as
  * every kernel above (also its self-check): C[M,N] fp32 = sum_k A[m,k] B[n,k]
  * with bf16 inputs and fp32 accumulation, each row of C bitwise independent of

@@ -259,3 +259,127 @@ def rlk_sum_ordered(parts, out=None, stream=None):
     arr = (ctypes.c_void_p * len(parts))(*[t.data_ptr() for t in parts])
     _check(_sum_fn(arr, len(parts), _ptr(out), n, _stream(stream)), "rlk_sum_ordered")
     return out
+
+
+_tp_fns = None
+
+
+def _tp():
+    global _tp_fns
+    if _tp_fns is None:
+        L = lib()
+        L.rlk_fwd_split_width.argtypes = []
+        L.rlk_fwd_split_width.restype = ctypes.c_int64
+        L.rlk_linear_logp_fwd_shard.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _I64,
+                                                ctypes.c_float, _P, _P, _P, _I64, _P, _P,
+                                                ctypes.c_size_t, _P]
+        L.rlk_linear_logp_fwd_shard.restype = ctypes.c_int
+        L.rlk_linear_logp_combine.argtypes = [_P, _P, _P, _I64, _I64, _P, _P, _I64, _I64, _P, _P,
+                                              _P, _P, ctypes.c_size_t, _P]
+        L.rlk_linear_logp_combine.restype = ctypes.c_int
+        L.rlk_bwd_chunk_width.argtypes = [_I64]
+        L.rlk_bwd_chunk_width.restype = ctypes.c_int64
+        L.rlk_linear_logp_bwd_shard.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _I64,
+                                                ctypes.c_float, _P, _P, _P, _P, _P, _I64, _I64,
+                                                _P, _P, ctypes.c_size_t, _P]
+        L.rlk_linear_logp_bwd_shard.restype = ctypes.c_int
+        L.rlk_dhidden_combine.argtypes = [_P, _I64, _I64, _P, _P]
+        L.rlk_dhidden_combine.restype = ctypes.c_int
+        _tp_fns = L
+    return _tp_fns
+
+
+def fwd_split_width() -> int:
+    """Vocab columns per forward split (shards must start at multiples of it)."""
+    return int(_tp().rlk_fwd_split_width())
+
+
+def rlk_linear_logp_fwd_shard(hidden, W_shard, targets, V, v0, temperature, part, ytgt,
+                              workspace=None, stream=None):
+    """Split triples of one vocab shard.  part: (part_m, part_s, part_b), each a
+    contiguous fp32 [T, Gs] tensor (Gs the same on every shard); ytgt: fp32 [T]
+    (rows with targets in the shard are written)."""
+    _req(hidden, torch.bfloat16, "hidden", 2)
+    _req(W_shard, torch.bfloat16, "W_shard", 2)
+    _req(targets, torch.int64, "targets", 1)
+    T, H = hidden.shape
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=hidden.device)
+    pm, ps, pb = part
+    for p in part:
+        _req(p, torch.float32, "part", 2)
+        if p.shape != pm.shape or p.shape[0] != T:
+            raise ValueError("part buffers must all be [T, Gs]")
+    _req(ytgt, torch.float32, "ytgt", 1)
+    _check(_tp().rlk_linear_logp_fwd_shard(_ptr(hidden), _ptr(W_shard), _ptr(targets), T, H, V,
+                                           v0, W_shard.shape[0], float(temperature), _ptr(pm),
+                                           _ptr(ps), _ptr(pb), pm.shape[1], _ptr(ytgt),
+                                           _ptr(workspace),
+                                           workspace.numel(), _stream(stream)),
+           "rlk_linear_logp_fwd_shard")
+    return workspace
+
+
+def rlk_linear_logp_combine(part, nshards, Gs, ytgt, targets, V, out=None, workspace=None,
+                            stream=None):
+    """logp, entropy, lse from split triples laid out [nshards][T][Gs]."""
+    T = targets.shape[0]
+    dev = targets.device
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = tuple(torch.empty(T, dtype=torch.float32, device=dev) for _ in range(3))
+    pm, ps, pb = part
+    logp, entropy, lse = out
+    _check(_tp().rlk_linear_logp_combine(_ptr(pm), _ptr(ps), _ptr(pb), nshards, Gs, _ptr(ytgt),
+                                         _ptr(targets), T, V, _ptr(logp), _ptr(entropy),
+                                         _ptr(lse), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)),
+           "rlk_linear_logp_combine")
+    return out
+
+
+def bwd_chunk_width(V: int) -> int:
+    """Vocab rows per backward chunk of a V-row head (shards of the backward
+    start at multiples of it)."""
+    return int(_tp().rlk_bwd_chunk_width(V))
+
+
+def rlk_linear_logp_bwd_shard(hidden, W_shard, targets, V, v0, temperature, lse, entropy, dlogp,
+                              dentropy, dh_parts, part_rows, dW_shard=None, workspace=None,
+                              stream=None):
+    """dW rows of one vocab shard and its per-chunk dHidden products.
+    dh_parts: contiguous fp32 [S, part_chunks, part_rows, H] (S = ceil(T /
+    part_rows)).  Returns (dW_shard, workspace)."""
+    _req(hidden, torch.bfloat16, "hidden", 2)
+    _req(W_shard, torch.bfloat16, "W_shard", 2)
+    _req(targets, torch.int64, "targets", 1)
+    _req(dh_parts, torch.float32, "dh_parts", 4)
+    T, H = hidden.shape
+    S, part_chunks, rows, Hp = dh_parts.shape
+    if rows != part_rows or Hp != H or S * part_rows < T:
+        raise ValueError("dh_parts must be [ceil(T/part_rows), part_chunks, part_rows, H]")
+    if dW_shard is None:
+        dW_shard = torch.empty(W_shard.shape[0], H, dtype=torch.float32, device=hidden.device)
+    if workspace is None:
+        workspace = make_workspace(T, H, V, True, hidden.device)
+    _check(_tp().rlk_linear_logp_bwd_shard(_ptr(hidden), _ptr(W_shard), _ptr(targets), T, H, V,
+                                           v0, W_shard.shape[0], float(temperature), _ptr(lse),
+                                           _ptr(entropy), _ptr(dlogp), _ptr(dentropy),
+                                           _ptr(dh_parts), part_rows, part_chunks,
+                                           _ptr(dW_shard), _ptr(workspace), workspace.numel(),
+                                           _stream(stream)),
+           "rlk_linear_logp_bwd_shard")
+    return dW_shard, workspace
+
+
+def rlk_dhidden_combine(dh_parts, nparts, out, stream=None):
+    """out (bf16, any shape) = the fixed-order sum of the first nparts blocks of
+    dh_parts (fp32, viewed as [blocks, out.numel()])."""
+    count = out.numel()
+    if not (dh_parts.is_contiguous() and dh_parts.dtype == torch.float32 and out.is_contiguous()
+            and out.dtype == torch.bfloat16 and dh_parts.numel() >= nparts * count):
+        raise ValueError("dh_parts: contiguous fp32 holding nparts blocks; out: contiguous bf16")
+    _check(_tp().rlk_dhidden_combine(_ptr(dh_parts), nparts, count, _ptr(out), _stream(stream)),
+           "rlk_dhidden_combine")
+    return out

@@ -214,37 +214,118 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
   return RLK_OK;
 }
 
-// Forward: pair-tile GEMM with the online epilogue, then the combine.
+// Forward, first half: the pair-tile GEMM over the `Vloc` rows of W (global
+// vocab rows v0 .. v0 + Vloc) with the online epilogue, writing one triple per
+// (row, 512-column split) to part_* ([T][ceil(Vloc / 512)]) and, for rows whose
+// target falls in these rows, the target's scaled logit to ytgt.
+rlk_status enqueue_fwd_partials(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                                int64_t T, int64_t H, int64_t Vloc, int64_t v0, float temperature,
+                                float* part_m, float* part_s, float* part_b, int64_t ldp,
+                                float* ytgt, uint32_t* err, cudaStream_t st) {
+  FwdArgs a;
+  if (!map_kmajor(&a.hid_k, hidden, H, T, H, kBM) || !map_kmajor(&a.w_k, W, H, Vloc, H, kBM))
+    return RLK_ERR_CUDA;
+  a.ep.targets = targets;
+  a.ep.part_m = part_m;
+  a.ep.part_s = part_s;
+  a.ep.part_b = part_b;
+  a.ep.ytgt = ytgt;
+  a.ep.T = static_cast<int>(T);
+  a.ep.V = static_cast<int>(Vloc);
+  a.ep.ldp = static_cast<int>(ldp);
+  a.ep.v0 = v0;
+  a.ep.scale_log2 = kLog2e / temperature;
+  a.err = err;
+  a.MT = static_cast<int>(ceil_div(T, kPairM));
+  a.NT = static_cast<int>(ceil_div(Vloc, kBN));
+  a.group = kFwdGroup;
+  a.NG = static_cast<int>(fwd_groups(Vloc));
+  a.KB = static_cast<int>(H / kBK);
+  a.total = static_cast<long long>(a.MT) * a.NG;
+  return launch_pair<kModeFwd>(a, a.total, false, st);
+}
+
+// Forward, second half: merge the splits (layout [nshards][T][Gs]) in global
+// split order.
+rlk_status enqueue_combine(const float* pm, const float* ps, const float* pb, int64_t Gs,
+                           const float* ytgt, const int64_t* targets, int64_t T, int64_t V,
+                           float* logp, float* entropy, float* lse, uint32_t* err,
+                           cudaStream_t st) {
+  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 8)), 256, 0, st>>>(
+      pm, ps, pb, ytgt, targets, static_cast<int>(T), static_cast<int>(V),
+      static_cast<int>(fwd_groups(V)), static_cast<int>(Gs), logp, entropy, lse, err);
+  return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
+}
+
 rlk_status enqueue_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
                        int64_t T, int64_t H, int64_t V, float temperature, float* logp,
                        float* entropy, float* lse, uint8_t* ws, const Layout& L,
                        cudaStream_t st) {
-  FwdArgs a;
-  if (!map_kmajor(&a.hid_k, hidden, H, T, H, kBM) || !map_kmajor(&a.w_k, W, H, V, H, kBM))
-    return RLK_ERR_CUDA;
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
-  a.ep.targets = targets;
-  a.ep.part_m = reinterpret_cast<float*>(ws + L.pm);
-  a.ep.part_s = reinterpret_cast<float*>(ws + L.ps);
-  a.ep.part_b = reinterpret_cast<float*>(ws + L.pb);
-  a.ep.ytgt = reinterpret_cast<float*>(ws + L.yt);
-  a.ep.T = static_cast<int>(T);
-  a.ep.V = static_cast<int>(V);
-  a.ep.G = static_cast<int>(fwd_groups(V));
-  a.ep.scale_log2 = kLog2e / temperature;
-  a.err = err;
-  a.MT = static_cast<int>(ceil_div(T, kPairM));
-  a.NT = static_cast<int>(ceil_div(V, kBN));
-  a.group = kFwdGroup;
-  a.NG = static_cast<int>(fwd_groups(V));
-  a.KB = static_cast<int>(H / kBK);
-  a.total = static_cast<long long>(a.MT) * a.NG;
-  rlk_status s = launch_pair<kModeFwd>(a, a.total, false, st);
+  float* pm = reinterpret_cast<float*>(ws + L.pm);
+  float* ps = reinterpret_cast<float*>(ws + L.ps);
+  float* pb = reinterpret_cast<float*>(ws + L.pb);
+  float* yt = reinterpret_cast<float*>(ws + L.yt);
+  rlk_status s = enqueue_fwd_partials(hidden, W, targets, T, H, V, 0, temperature, pm, ps, pb,
+                                      fwd_groups(V), yt, err, st);
   if (s != RLK_OK) return s;
-  combine_kernel<<<static_cast<unsigned>(ceil_div(T, 8)), 256, 0, st>>>(
-      a.ep.part_m, a.ep.part_s, a.ep.part_b, a.ep.ytgt, targets, static_cast<int>(T),
-      static_cast<int>(V), a.NG, logp, entropy, lse, err);
-  return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
+  return enqueue_combine(pm, ps, pb, fwd_groups(V), yt, targets, T, V, logp, entropy, lse, err,
+                         st);
+}
+
+// Backward over W rows [v0, v0 + Vloc) of a Vfull-row head (the whole head:
+// v0 = 0, Vloc = Vfull), chunked as the full head is.  dh_parts null: dHidden
+// accumulated over the chunks and written as bf16; else each chunk's fp32
+// product goes to dh_parts (EpiDh::kPart layout).
+rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
+                       int64_t T, int64_t H, int64_t Vloc, int64_t v0, int64_t Vfull,
+                       float temperature, const float* lse, const float* entropy,
+                       const float* dlogp, const float* dentropy, rlk_bf16* dHidden,
+                       float* dh_parts, int64_t part_rows, int64_t part_chunks, float* dW,
+                       uint8_t* ws, const Layout& L, cudaStream_t st) {
+  BwdParams P;
+  P.plan = make_bwd_plan(T, H, Vloc, vchunk(Vfull));
+  const BwdPlan& pl = P.plan;
+  if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
+      !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM) || !map_mnmajor(&P.maps.w_mn, W, H, Vloc, H) ||
+      !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
+    return RLK_ERR_CUDA;
+  for (int i = 0; i < kDxBuffers; ++i) {
+    P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
+    if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
+        !map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx) ||
+        !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return RLK_ERR_CUDA;
+  }
+  P.targets = targets;
+  P.lse = lse;
+  P.entropy = entropy;
+  P.dlogp = dlogp;
+  P.dentropy = dentropy;
+  P.dh_acc = reinterpret_cast<float*>(ws + L.dh);
+  P.dhidden = reinterpret_cast<__nv_bfloat16*>(dHidden);
+  P.dh_parts = dh_parts;
+  P.part_rows = static_cast<int>(part_rows);
+  P.part_chunks = static_cast<int>(part_chunks);
+  P.v0 = v0;
+  P.Vfull = Vfull;
+  P.dW = dW;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
+  const size_t nc = static_cast<size_t>(pl.NC);
+  P.rdone_m = cnt;
+  P.rdone_j = P.rdone_m + nc * pl.MT;
+  P.hdone = P.rdone_j + nc * pl.RT_full;
+  P.bufdone = P.hdone + nc * pl.MT * pl.NH;
+  P.next_unit = P.bufdone + nc;
+  P.err = reinterpret_cast<uint32_t*>(ws);
+  P.scale_log2 = kLog2e / temperature;
+  P.inv_tau = 1.0f / temperature;
+
+  if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
+  // Units wait on units claimed earlier, and only running CTA pairs claim
+  // units, so no pair ever waits on one that has not started: the launch needs
+  // no co-residency guarantee.
+  return launch_pair<kModeBwd>(P, pl.total, false, st);
 }
 
 }  // namespace
@@ -314,45 +395,10 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   if (workspace_bytes < L.bwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device(&sms)) != RLK_OK) return s;
 
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  BwdParams P;
-  P.plan = bwd_plan(T, H, V);
-  const BwdPlan& pl = P.plan;
-  if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
-      !map_kmajor(&P.maps.w_k, W, H, V, H, kBM) || !map_mnmajor(&P.maps.w_mn, W, H, V, H) ||
-      !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
-    return RLK_ERR_CUDA;
-  for (int i = 0; i < kDxBuffers; ++i) {
-    P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
-    if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx) ||
-        !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return RLK_ERR_CUDA;
-  }
-  P.targets = targets;
-  P.lse = lse;
-  P.entropy = entropy;
-  P.dlogp = dlogp;
-  P.dentropy = dentropy;
-  P.dh_acc = reinterpret_cast<float*>(ws + L.dh);
-  P.dhidden = reinterpret_cast<__nv_bfloat16*>(dHidden);
-  P.dW = dW;
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(ws + L.cnt);
-  const size_t nc = static_cast<size_t>(pl.NC);
-  P.rdone_m = cnt;
-  P.rdone_j = P.rdone_m + nc * pl.MT;
-  P.hdone = P.rdone_j + nc * pl.RT_full;
-  P.bufdone = P.hdone + nc * pl.MT * pl.NH;
-  P.next_unit = P.bufdone + nc;
-  P.err = reinterpret_cast<uint32_t*>(ws);
-  P.scale_log2 = kLog2e / temperature;
-  P.inv_tau = 1.0f / temperature;
-
-  if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
-  // Units wait on units claimed earlier, and only running CTA pairs claim
-  // units, so no pair ever waits on one that has not started: the launch needs
-  // no co-residency guarantee.
-  if ((s = launch_pair<kModeBwd>(P, pl.total, false, st)) != RLK_OK) return s;
+  if ((s = enqueue_bwd(hidden, W, targets, T, H, V, 0, V, temperature, lse, entropy, dlogp,
+                       dentropy, dHidden, nullptr, 0, 0, dW, static_cast<uint8_t*>(workspace), L,
+                       st)) != RLK_OK)
+    return s;
   g_calls[1].fetch_add(1);
   return RLK_OK;
 }
@@ -435,6 +481,164 @@ const char* rlk_status_string(rlk_status status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Vocab-parallel (tensor-parallel) forward: shards of W whose first rows are
+// aligned to the 512-column splits produce exactly the single-GPU split
+// triples, and the combine merges them in global split order.
+// ---------------------------------------------------------------------------
+extern "C" int64_t rlk_fwd_split_width(void) { return static_cast<int64_t>(kBN) * kFwdGroup; }
+
+extern "C" rlk_status rlk_linear_logp_fwd_shard(const rlk_bf16* hidden, const rlk_bf16* W_shard,
+                                                const int64_t* targets, int64_t T, int64_t H,
+                                                int64_t V, int64_t v0, int64_t V_shard,
+                                                float temperature, float* part_m, float* part_s,
+                                                float* part_b, int64_t Gs, float* ytgt,
+                                                void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (v0 < 0 || V_shard < 1 || v0 + V_shard > V) return RLK_ERR_INVALID_ARG;
+  if (Gs < fwd_groups(V_shard) || Gs > fwd_groups(V)) return RLK_ERR_INVALID_ARG;
+  // splits must not straddle shards: every shard but the last is whole splits
+  if (v0 % rlk_fwd_split_width() != 0 || (v0 + V_shard != V && V_shard % rlk_fwd_split_width()))
+    return RLK_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return RLK_OK;
+  if (!hidden || !W_shard || !targets || !part_m || !part_s || !part_b || !ytgt || !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W_shard, 16) || !aligned(workspace, 256) ||
+      !aligned(targets, 8) || !aligned(part_m, 4) || !aligned(part_s, 4) || !aligned(part_b, 4) ||
+      !aligned(ytgt, 4))
+    return RLK_ERR_MISALIGNED;
+  if (workspace_bytes < kHeader) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  return enqueue_fwd_partials(hidden, W_shard, targets, T, H, V_shard, v0, temperature, part_m,
+                              part_s, part_b, Gs, ytgt, static_cast<uint32_t*>(workspace),
+                              static_cast<cudaStream_t>(stream));
+}
+
+extern "C" rlk_status rlk_linear_logp_combine(const float* part_m, const float* part_s,
+                                              const float* part_b, int64_t nshards, int64_t Gs,
+                                              const float* ytgt, const int64_t* targets,
+                                              int64_t T, int64_t V, float* logp, float* entropy,
+                                              float* lse, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  rlk_status s = check_sizes(T, 64, V, 1.0f);
+  if (s != RLK_OK) return s;
+  const int64_t G = fwd_groups(V);
+  if (nshards < 1 || Gs < 1 || (nshards - 1) * Gs >= G || nshards * Gs < G)
+    return RLK_ERR_INVALID_ARG;
+  if (T == 0) return RLK_OK;
+  if (!part_m || !part_s || !part_b || !ytgt || !targets || !logp || !entropy || !lse ||
+      !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(targets, 8) || !aligned(part_m, 4) ||
+      !aligned(part_s, 4) || !aligned(part_b, 4) || !aligned(ytgt, 4) || !aligned(logp, 4) ||
+      !aligned(entropy, 4) || !aligned(lse, 4))
+    return RLK_ERR_MISALIGNED;
+  if (workspace_bytes < kHeader) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  return enqueue_combine(part_m, part_s, part_b, Gs, ytgt, targets, T, V, logp, entropy, lse,
+                         static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+// Vocab-parallel backward.  A shard's chunks are the full head's chunks
+// (boundaries at multiples of rlk_bwd_chunk_width(V)), so its recompute,
+// dlogits, per-chunk dHidden products and dW rows are bit for bit those of the
+// single-GPU backward; rlk_dhidden_combine then adds the chunks' products in
+// global chunk order with the same fp32 additions and bf16 rounding.
+extern "C" int64_t rlk_bwd_chunk_width(int64_t V) {
+  if (V <= 0 || V >= (int64_t{1} << 31)) return 0;
+  return vchunk(V);
+}
+
+extern "C" rlk_status rlk_linear_logp_bwd_shard(
+    const rlk_bf16* hidden, const rlk_bf16* W_shard, const int64_t* targets, int64_t T, int64_t H,
+    int64_t V, int64_t v0, int64_t V_shard, float temperature, const float* lse,
+    const float* entropy, const float* dlogp, const float* dentropy, float* dh_parts,
+    int64_t part_rows, int64_t part_chunks, float* dW_shard, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (v0 < 0 || V_shard < 1 || v0 + V_shard > V) return RLK_ERR_INVALID_ARG;
+  const int64_t vc = vchunk(V);
+  if (v0 % vc != 0 || (v0 + V_shard != V && V_shard % vc != 0)) return RLK_ERR_UNSUPPORTED_SHAPE;
+  if (part_rows < 1 || part_rows >= (int64_t{1} << 31) || part_chunks < ceil_div(V_shard, vc) ||
+      part_chunks > ceil_div(V, vc))
+    return RLK_ERR_INVALID_ARG;
+  if (!dW_shard) return RLK_ERR_INVALID_ARG;
+  if (!aligned(dW_shard, 16)) return RLK_ERR_MISALIGNED;
+  int sms = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if ((s = check_device(&sms)) != RLK_OK) return s;
+    return cudaMemsetAsync(dW_shard, 0, static_cast<size_t>(V_shard) * H * 4, st) == cudaSuccess
+               ? RLK_OK
+               : RLK_ERR_CUDA;
+  }
+  if (!hidden || !W_shard || !targets || !lse || !entropy || !dlogp || !dentropy || !dh_parts ||
+      !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W_shard, 16) || !aligned(dh_parts, 16) ||
+      !aligned(workspace, 256) || !aligned(targets, 8) || !aligned(lse, 4) ||
+      !aligned(entropy, 4) || !aligned(dlogp, 4) || !aligned(dentropy, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);  // sized for the full head: covers any shard
+  if (workspace_bytes < L.bwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  return enqueue_bwd(hidden, W_shard, targets, T, H, V_shard, v0, V, temperature, lse, entropy,
+                     dlogp, dentropy, nullptr, dh_parts, part_rows, part_chunks, dW_shard,
+                     static_cast<uint8_t*>(workspace), L, st);
+}
+
+namespace rlk {
+namespace {
+
+// out[i] = bf16(((p_0[i] + p_1[i]) + p_2[i]) + ...), the same fp32 additions
+// (old + new) and rounding as the dHidden epilogue's chunk chain.
+__global__ void __launch_bounds__(256) dhidden_combine_kernel(const float* __restrict__ parts,
+                                                              int nparts, int64_t count,
+                                                              __nv_bfloat16* __restrict__ out) {
+  const int64_t n4 = count / 4;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += stride) {
+    float4 a = reinterpret_cast<const float4*>(parts)[i];
+    for (int k = 1; k < nparts; ++k) {
+      const float4 v = reinterpret_cast<const float4*>(parts + k * count)[i];
+      a.x = a.x + v.x;
+      a.y = a.y + v.y;
+      a.z = a.z + v.z;
+      a.w = a.w + v.w;
+    }
+    uint2 w;
+    w.x = pack_bf16x2(a.x, a.y);
+    w.y = pack_bf16x2(a.z, a.w);
+    reinterpret_cast<uint2*>(out)[i] = w;
+  }
+}
+
+}  // namespace
+}  // namespace rlk
+
+extern "C" rlk_status rlk_dhidden_combine(const float* dh_parts, int64_t nparts, int64_t count,
+                                          rlk_bf16* out, void* stream) {
+  if (nparts < 1 || nparts > (int64_t{1} << 20) || count < 0) return RLK_ERR_INVALID_ARG;
+  if (count % 4) return RLK_ERR_UNSUPPORTED_SHAPE;
+  if (count == 0) return RLK_OK;
+  if (!dh_parts || !out) return RLK_ERR_INVALID_ARG;
+  if (!aligned(dh_parts, 16) || !aligned(out, 8)) return RLK_ERR_MISALIGNED;
+  int sms = 0;
+  rlk_status s = check_device(&sms);
+  if (s != RLK_OK) return s;
+  const int64_t blocks = std::min<int64_t>(ceil_div(count / 4, 256), static_cast<int64_t>(sms) * 8);
+  dhidden_combine_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                           static_cast<cudaStream_t>(stream)>>>(
+      dh_parts, static_cast<int>(nparts), count, reinterpret_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError() == cudaSuccess ? RLK_OK : RLK_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------------------
 // Fixed-order sum of equally shaped fp32 buffers (the data-parallel exchange

@@ -66,6 +66,11 @@ struct BwdParams {
   __nv_bfloat16* dx[kDxBuffers];
   float* dh_acc;
   __nv_bfloat16* dhidden;
+  float* dh_parts;    // non-null: per-chunk dHidden products instead (EpiDh::kPart)
+  int part_rows;
+  int part_chunks;
+  int64_t v0;         // global vocab index of W's first row (a vocab shard's offset)
+  int64_t Vfull;      // full vocabulary
   float* dW;
   uint32_t* rdone_m;  // [NC][MT]
   uint32_t* rdone_j;  // [NC][RT_full]

@@ -46,13 +46,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 struct EpiFwd {
   struct Params {
     const int64_t* targets;
-    float* part_m;  // [T][G] (row-major: a row's splits are contiguous)
+    float* part_m;  // [T][ldp] (row-major: a row's splits are contiguous)
     float* part_s;
     float* part_b;
     float* ytgt;
     int T;
-    int V;
-    int G;             // vocab splits
+    int V;             // vocab columns of this W (a shard's own count for a shard)
+    int ldp;           // row stride of part_*: at least this W's vocab splits
+    int64_t v0;        // global vocab index of this W's first row (0 unless a shard)
     float scale_log2;  // log2(e) / tau
   };
   struct State {
@@ -65,7 +66,7 @@ struct EpiFwd {
   __device__ static void begin_unit(const Params& p, State& st, int row, int, int) {
     st.row = row;
     st.valid = row < p.T;
-    st.tgt = st.valid ? p.targets[row] : -1;
+    st.tgt = st.valid ? p.targets[row] - p.v0 : -1;  // local column of the target
     st.m = kMaskLogit;
     st.s = 0.f;
     st.b = 0.f;
@@ -112,7 +113,7 @@ struct EpiFwd {
 
   __device__ static void end_unit(const Params& p, State& st, int g) {
     if (st.valid) {
-      const size_t i = static_cast<size_t>(st.row) * p.G + g;
+      const size_t i = static_cast<size_t>(st.row) * p.ldp + g;
       p.part_m[i] = st.m;
       p.part_s[i] = st.s;
       p.part_b[i] = st.b;
@@ -134,9 +135,11 @@ struct EpiDlogits {
     __nv_bfloat16* dX;
     uint32_t* err;
     int T;
-    int V;
+    int V;             // vocab rows of this W (a shard's own count for a shard)
     int c0;
     int ldx;
+    int64_t v0;        // global vocab index of this W's first row (0 unless a shard)
+    int64_t Vfull;     // full vocabulary (targets are global indices)
     float scale_log2;  // log2(e) / tau
     float inv_tau;
   };
@@ -163,8 +166,9 @@ struct EpiDlogits {
       st.k1 = p.inv_tau * (dl - de * ez);
       st.k2 = p.inv_tau * de * kLn2;
       st.hot = p.inv_tau * dl;
-      if (tg >= 0 && tg < p.V) {
-        st.tloc = tg - p.c0;
+      if (tg >= 0 && tg < p.Vfull) {
+        const int64_t t = tg - p.v0;  // shard-local; the target is elsewhere if out of [0, V)
+        if (t >= 0 && t < p.V) st.tloc = t - p.c0;
       } else if (p.c0 == 0) {
         atomicOr(p.err, kDevErrTarget);
       }
@@ -229,24 +233,36 @@ struct EpiDlogits {
 
 // dHidden: acc[T,H] (fp32 workspace) collects the vocab chunks in ascending
 // order: chunk 0 stores, later chunks add (old + new), the last chunk writes
-// the bf16 result.
+// the bf16 result.  kPart instead stores chunk c's own fp32 product into a
+// parts buffer laid out [row slice s][chunk c][row r][H] (row = s * part_rows
+// + r), for a sum in global chunk order elsewhere.
 struct EpiDh {
-  enum Mode { kFirst = 0, kMiddle = 1, kLast = 2, kOnly = 3 };
+  enum Mode { kFirst = 0, kMiddle = 1, kLast = 2, kOnly = 3, kPart = 4 };
   struct Params {
-    float* acc;
+    float* acc;  // [T][H], or the parts buffer for kPart
     __nv_bfloat16* out;
     int T;
     int H;
     int mode;
+    int c;            // kPart: the chunk
+    int part_rows;    // kPart: rows per slice
+    int part_chunks;  // kPart: chunk slots per slice
   };
   struct State {
-    int row;
+    float* arow;
+    __nv_bfloat16* orow;
     bool valid;
   };
 
   __device__ static void begin_unit(const Params& p, State& st, int row, int, int) {
-    st.row = row;
     st.valid = row < p.T;
+    size_t a = static_cast<size_t>(row) * p.H;
+    if (p.mode == kPart) {
+      const int s = row / p.part_rows, r = row - s * p.part_rows;
+      a = ((static_cast<size_t>(s) * p.part_chunks + p.c) * p.part_rows + r) * p.H;
+    }
+    st.arow = p.acc + a;
+    st.orow = p.out + static_cast<size_t>(row) * p.H;
   }
 
   __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt) {
@@ -260,8 +276,7 @@ struct EpiDh {
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-      const size_t off = static_cast<size_t>(st.row) * p.H + col0;
-      float4* pa = reinterpret_cast<float4*>(p.acc + off);
+      float4* pa = reinterpret_cast<float4*>(st.arow + col0);
       if (p.mode == kMiddle || p.mode == kLast) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -272,12 +287,12 @@ struct EpiDh {
           v[4 * q + 3] = o.w + v[4 * q + 3];
         }
       }
-      if (p.mode == kFirst || p.mode == kMiddle) {
+      if (p.mode == kFirst || p.mode == kMiddle || p.mode == kPart) {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           pa[q] = make_float4(v[4 * q + 0], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       } else {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + off);
+        uint4* dst = reinterpret_cast<uint4*>(st.orow + col0);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 w;
@@ -360,20 +375,26 @@ __device__ __forceinline__ Triple merge_triple(Triple x, Triple y) {
   return r;
 }
 
+// Partials are laid out [shard][T][Gs]: split g of row t sits in shard g / Gs
+// at local split g % Gs (one shard of Gs = G splits without tensor
+// parallelism).  The merge order depends only on G.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ pm,
                                                       const float* __restrict__ ps,
                                                       const float* __restrict__ pb,
                                                       const float* __restrict__ ytgt,
                                                       const int64_t* __restrict__ targets, int T,
-                                                      int V, int G, float* __restrict__ logp,
+                                                      int V, int G, int Gs,
+                                                      float* __restrict__ logp,
                                                       float* __restrict__ entropy,
                                                       float* __restrict__ lse, uint32_t* err) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;  // warp-uniform
-  const size_t base = static_cast<size_t>(t) * G;
   Triple acc{kMaskLogit, 0.f, 0.f};
-  for (int g = lane; g < G; g += 32) acc = merge_triple(acc, Triple{pm[base + g], ps[base + g], pb[base + g]});
+  for (int g = lane; g < G; g += 32) {
+    const size_t i = (static_cast<size_t>(g / Gs) * T + t) * Gs + g % Gs;
+    acc = merge_triple(acc, Triple{pm[i], ps[i], pb[i]});
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     Triple o;

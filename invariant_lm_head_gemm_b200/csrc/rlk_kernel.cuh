@@ -488,6 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.V = pl.V;
             p.c0 = j.c * pl.ldx;
             p.ldx = pl.ldx;
+            p.v0 = P.v0;
+            p.Vfull = P.Vfull;
             p.scale_log2 = P.scale_log2;
             p.inv_tau = P.inv_tau;
             EpiDlogits::State st;
@@ -500,10 +502,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.out = P.dhidden;
             p.T = pl.T;
             p.H = pl.H;
-            p.mode = pl.NC == 1          ? EpiDh::kOnly
+            p.mode = P.dh_parts          ? EpiDh::kPart
+                     : pl.NC == 1        ? EpiDh::kOnly
                      : j.c == 0          ? EpiDh::kFirst
                      : j.c == pl.NC - 1  ? EpiDh::kLast
                                          : EpiDh::kMiddle;
+            if (P.dh_parts) p.acc = P.dh_parts;
+            p.c = j.c;
+            p.part_rows = P.part_rows;
+            p.part_chunks = P.part_chunks;
             EpiDh::State st;
             EpiDh::begin_unit(p, st, row, 0, 0);
             EpiDh::tile(p, st, taddr, j.nt);

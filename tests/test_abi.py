@@ -123,4 +123,79 @@ def test_valid_call_without_a_gpu_is_refused(L):
     assert _bwd(L) == DEVICE
     assert _bwd(L, T=0) == DEVICE
     assert L.rlk_gemm_bf16_f32(A16, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == DEVICE
+    assert _shard(L) == DEVICE and _combine(L) == DEVICE
+    assert _bshard(L) == DEVICE and L.rlk_dhidden_combine(A16, 2, 8, A16, None) == DEVICE
     assert binding.call_count(0) == 0 and binding.call_count(1) == 0
+
+
+def _shard(L, v0=0, Vs=512, Gs=1, V=2000, T=4, H=64, tau=1.0, pm=A16, ytgt=A16, ws=A256,
+           wsb=256, hidden=A16):
+    binding._tp()
+    return L.rlk_linear_logp_fwd_shard(hidden, A16, A16, T, H, V, v0, Vs, tau, pm, A16, A16, Gs,
+                                       ytgt, ws, wsb, None)
+
+
+def _combine(L, nshards=2, Gs=2, V=2000, T=4, pm=A16, ws=A256, wsb=256, lse=A16):
+    binding._tp()
+    return L.rlk_linear_logp_combine(pm, A16, A16, nshards, Gs, A16, A16, T, V, A16, A16, lse, ws,
+                                     wsb, None)
+
+
+def test_tp_argument_errors(L):
+    assert L.rlk_fwd_split_width() == 512
+    assert _shard(L, v0=100) == SHAPE              # shard off a split boundary
+    assert _shard(L, v0=1536, Vs=512) == INVALID   # past V = 2000
+    assert _shard(L, Vs=0) == INVALID
+    assert _shard(L, v0=-512) == INVALID
+    assert _shard(L, Vs=1024, Gs=1) == INVALID     # row stride below the shard's splits
+    assert _shard(L, Gs=5) == INVALID              # row stride above the vocab's splits
+    assert _shard(L, H=96) == SHAPE
+    assert _shard(L, tau=0.0) == INVALID
+    assert _shard(L, T=0, hidden=None) == OK
+    assert _shard(L, hidden=None) == INVALID
+    assert _shard(L, pm=A16 + 2) == MISALIGNED
+    assert _shard(L, wsb=255) == WS_SMALL
+    # (nshards - 1) * Gs < ceil(V / 512) <= nshards * Gs
+    assert _combine(L, nshards=1, Gs=3) == INVALID
+    assert _combine(L, nshards=3, Gs=2) == INVALID
+    assert _combine(L, nshards=0) == INVALID
+    assert _combine(L, lse=None) == INVALID
+    assert _combine(L, pm=A16 + 1) == MISALIGNED
+    assert _combine(L, ws=A256 + 8) == MISALIGNED
+    assert _combine(L, wsb=100) == WS_SMALL
+    assert _combine(L, T=0) == OK
+
+
+def _bshard(L, v0=0, Vs=8192, V=20000, T=4, H=64, R=4, cps=2, dW=A16, parts=A16, ws=A256,
+            wsb=1 << 30, hidden=A16):
+    binding._tp()
+    return L.rlk_linear_logp_bwd_shard(hidden, A16, A16, T, H, V, v0, Vs, 1.0, A16, A16, A16, A16,
+                                       parts, R, cps, dW, ws, wsb, None)
+
+
+def test_tp_backward_argument_errors(L):
+    binding._tp()
+    assert L.rlk_bwd_chunk_width(20000) == 8192
+    assert L.rlk_bwd_chunk_width(1537) == 1792
+    assert L.rlk_bwd_chunk_width(0) == 0
+    assert _bshard(L, v0=512) == SHAPE               # off the 8192-row chunk grid
+    assert _bshard(L, Vs=9000) == SHAPE              # not the last shard, not whole chunks
+    assert _bshard(L, v0=16384, Vs=3616, cps=1) != SHAPE   # the ragged last shard is fine
+    assert _bshard(L, v0=16384, Vs=8192) == INVALID  # past V
+    assert _bshard(L, R=0) == INVALID
+    assert _bshard(L, Vs=16384, cps=1) == INVALID    # fewer slots than the shard's chunks
+    assert _bshard(L, cps=4) == INVALID              # more slots than the head has chunks
+    assert _bshard(L, dW=None) == INVALID
+    assert _bshard(L, dW=A16 + 4) == MISALIGNED
+    assert _bshard(L, parts=None) == INVALID
+    assert _bshard(L, parts=A16 + 8) == MISALIGNED
+    assert _bshard(L, H=96) == SHAPE
+    need = binding.workspace_bytes(4, 64, 20000, True)
+    assert _bshard(L, wsb=need - 1) == WS_SMALL
+    c = L.rlk_dhidden_combine
+    assert c(A16, 0, 8, A16, None) == INVALID
+    assert c(A16, 2, 6, A16, None) == SHAPE
+    assert c(A16, 2, 0, A16, None) == OK
+    assert c(None, 2, 8, A16, None) == INVALID
+    assert c(A16 + 4, 2, 8, A16, None) == MISALIGNED
+    assert c(A16, 2, 8, A16 + 2, None) == MISALIGNED

@@ -102,3 +102,131 @@ def test_dw_reduce_scatter_is_the_rank_ordered_sum(world, V):
         assert np.array_equal(got.view(np.uint32), full[r0:r1].numpy().view(np.uint32))
         covered += r1 - r0
     assert covered == V
+
+
+def _tp_worker(rank, world, port, V, T, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from invariant_lm_head_gemm_b200 import binding, tp
+    # stand-ins for the CUDA entry points: record what the glue hands over
+    seen = {}
+
+    def fake_shard(hidden, W_shard, targets, V_, v0, temperature, part, ytgt, workspace=None,
+                   stream=None):
+        for k, p in enumerate(part):
+            p.copy_(torch.full_like(p, 100 * rank + k))
+        owned = (targets >= v0) & (targets < v0 + W_shard.shape[0])
+        ytgt[owned] = targets[owned].float()
+
+    def fake_combine(part, nshards, Gs, ytgt, targets, V_, out=None, workspace=None, stream=None):
+        seen.update(nshards=nshards, Gs=Gs, part=[p.clone() for p in part], ytgt=ytgt.clone())
+        return None
+
+    binding.fwd_split_width = lambda: 512
+    binding.bwd_chunk_width = lambda V_: 8192
+    binding.rlk_linear_logp_fwd_shard = fake_shard
+    binding.rlk_linear_logp_combine = fake_combine
+    v0, v1 = tp.shard_rows(V, world, rank, tp.shard_alignment(V))
+    targets = torch.arange(T, dtype=torch.int64) * (V // T)
+    tp.tp_linear_logp_fwd(torch.zeros(T, 64), torch.zeros(v1 - v0, 64), targets, V, 1.0)
+    out[rank] = (v0, v1, seen["nshards"], seen["Gs"],
+                 [p[:, 0, 0].tolist() for p in seen["part"]], seen["ytgt"].tolist())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_tp_glue_gathers_shards_in_rank_order():
+    world, V, T = 3, 151936, 6
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_tp_worker, args=(world, _free_port(), V, T, out), nprocs=world, join=True)
+        res = dict(out)
+    bounds = [res[r][:2] for r in range(world)]
+    assert bounds[0][0] == 0 and bounds[-1][1] == V
+    assert all(b[0] % 8192 == 0 for b in bounds)
+    assert all(bounds[r][1] == bounds[r + 1][0] for r in range(world - 1))
+    for r in range(world):
+        _, _, nshards, Gs, parts, ytgt = res[r]
+        assert nshards == world and (nshards - 1) * Gs < -(-V // 512) <= nshards * Gs
+        for k in range(3):                       # shard r's triples at position r
+            assert parts[k] == [100 * q + k for q in range(world)]
+        assert ytgt == [float(t * (V // T)) for t in range(T)]   # every row owned once
+
+
+def _tp_bwd_worker(rank, world, port, V, T, H, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from invariant_lm_head_gemm_b200 import binding, tp
+    seen = {}
+
+    def fake_bwd_shard(hidden, W_shard, targets, V_, v0, tau, lse, ent, dl, de, parts, R,
+                       dW_shard=None, workspace=None, stream=None):
+        # value = 1000 * rank + 100 * slice + 10 * local chunk + local row
+        S, cps, R_, H_ = parts.shape
+        nloc = -(-W_shard.shape[0] // 8192)
+        for s in range(S):
+            for k in range(nloc):
+                for r in range(R_):
+                    parts[s, k, r] = 1000 * rank + 100 * s + 10 * k + r
+        return torch.full((W_shard.shape[0], H_), float(rank)), None
+
+    def fake_combine(parts, nparts, out, stream=None):
+        seen.update(nparts=nparts, recv=parts.clone())
+        out.copy_(torch.full_like(out, rank))
+        return out
+
+    binding.fwd_split_width = lambda: 512
+    binding.bwd_chunk_width = lambda V_: 8192
+    binding.rlk_linear_logp_bwd_shard = fake_bwd_shard
+    binding.rlk_dhidden_combine = fake_combine
+    v0, v1 = tp.shard_rows(V, world, rank, tp.shard_alignment(V))
+    z = torch.zeros(T)
+    dH, dW = tp.tp_linear_logp_bwd(torch.zeros(T, H, dtype=torch.bfloat16),
+                                   torch.zeros(v1 - v0, H), torch.zeros(T, dtype=torch.int64), V,
+                                   1.0, z, z, z, z)
+    out[rank] = (v0, v1, seen["nparts"], seen["recv"][:, :, :, 0].tolist(),
+                 dH[:, 0].float().tolist(), list(dW.shape))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,V,T", [(3, 40000, 7), (2, 151936, 4), (4, 20000, 3)])
+def test_tp_backward_glue_routes_chunk_products(world, V, T):
+    H = 4
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_tp_bwd_worker, args=(world, _free_port(), V, T, H, out), nprocs=world,
+                 join=True)
+        res = dict(out)
+    R = -(-T // world)
+    nchunks = -(-V // 8192)
+    owners = []          # (rank, local chunk) of every global chunk, in order
+    for r in range(world):
+        v0, v1 = res[r][:2]
+        assert v1 == v0 or (v0 % 8192 == 0 and (v1 == V or (v1 - v0) % 8192 == 0))
+        owners += [(r, k) for k in range(-(-(v1 - v0) // 8192))]
+        assert res[r][5] == [v1 - v0, H]
+    assert len(owners) == nchunks
+    for q in range(world):
+        _, _, nparts, recv, dH, _ = res[q]
+        assert nparts == nchunks
+        cps = len(recv[0])
+        flat = [recv[src][k] for src in range(world) for k in range(cps)]
+        # the first nchunks blocks are the chunks in global order, each holding
+        # row slice q of its owner's product
+        for g, (src, k) in enumerate(owners):
+            assert flat[g] == [1000 * src + 100 * q + 10 * k + r for r in range(R)], (q, g)
+        # dHidden rows come back in rank order, the padding rows dropped
+        assert dH == [float(t // R) for t in range(T)]
