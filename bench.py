@@ -278,6 +278,56 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
+    # ---------------------------------------------------------------- decode-shaped forward
+    # Rollout scoring / decode: the first T rows of the batch against the same
+    # W (1.245 GB, far above L2, so every call streams W from HBM).  Bound by
+    # HBM: algorithmic bytes = W + hidden rows + targets + outputs.  Timed as
+    # CUDA-graph replays of one captured call, the way a decode loop runs it
+    # (an eager call at these sizes is bound by the host's launch work; its
+    # time is reported too), before the long GEMM steps drive the clocks down
+    # to the power cap.  One untimed pass over the sizes first.
+    def decode_us(Td):
+        h_d, t_d = hid[:Td].contiguous(), tg[:Td].contiguous()
+        outs = tuple(torch.empty(Td, device=dev) for _ in range(3))
+
+        def call():
+            binding.rlk_linear_logp_fwd(h_d, W, t_d, 1.0, ws, out=outs)
+
+        call()
+        torch.cuda.synchronize()
+        e_a = torch.cuda.Event(enable_timing=True)
+        e_b = torch.cuda.Event(enable_timing=True)
+        e_a.record(stream)
+        for _ in range(10):
+            call()
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        eager = 1e3 * e_a.elapsed_time(e_b) / 10
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        for _ in range(3):
+            graph.replay()
+        e_a.record(stream)
+        for _ in range(20):
+            graph.replay()
+        e_b.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * e_a.elapsed_time(e_b) / 20, eager
+
+    decode_rows = (1, 4, 16, 64, 128, 256)
+    for Td in decode_rows:
+        decode_us(Td)
+    dec_us = [decode_us(Td) for Td in decode_rows]
+    dec_gbs = [(V * H * 2 + Td * (H * 2 + 8 + 12)) / (u * 1e-6) / 1e9
+               for Td, (u, _) in zip(decode_rows, dec_us)]
+    decode = {"kernel": "decode_fwd_kernel (T <= 128: operands swapped, M = 128 vocab rows, "
+                        "N = T padded to 16/32) + combine; larger T: the pair kernel",
+              "bound": "hbm", "unit": "GB/s", "timing": "CUDA-graph replay, 20 calls",
+              "rows": list(decode_rows), "us_per_call": [u for u, _ in dec_us],
+              "eager_us_per_call": [e for _, e in dec_us], "achieved": dec_gbs,
+              "frac": [g / peaks()[0]["hbm_gbs"] for g in dec_gbs]}
+
     # ---------------------------------------------------------------- device-resident
     for _ in range(args.warmup):
         step()
@@ -313,6 +363,32 @@ def run_ours(args):
                                                              out=(logp, ent, lse)), args.steps)
     bwd_ms = per_call_ms(lambda: binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent, dl, de,
                                                              ws, out=(dH, dW)), args.steps)
+
+    # ---------------------------------------------------------------- one rank of TP = 8
+    # Vocab-parallel: rank 0's shard (W rows [0, 24576)) on the same batch;
+    # kernels only (the exchange needs the other ranks).
+    from invariant_lm_head_gemm_b200 import tp as tpmod
+    tp_world = 8
+    align = tpmod.shard_alignment(V)
+    s0, s1 = tpmod.shard_rows(V, tp_world, 0, align)
+    W_s = W[s0:s1]
+    Gs = -(-(s1 - s0) // binding.fwd_split_width())
+    tp_part = [torch.empty(T, Gs, device=dev) for _ in range(3)]
+    tp_yt = torch.empty(T, device=dev)
+    R = -(-T // tp_world)
+    cps = -(-(s1 - s0) // binding.bwd_chunk_width(V))
+    tp_dh = torch.empty(tp_world, cps, R, H, device=dev)
+    tp_dW = torch.empty(s1 - s0, H, device=dev)
+    tp_f = per_call_ms(lambda: binding.rlk_linear_logp_fwd_shard(hid, W_s, tg, V, s0, 1.0, tp_part,
+                                                                tp_yt, ws), args.steps)
+    tp_b = per_call_ms(lambda: binding.rlk_linear_logp_bwd_shard(
+        hid, W_s, tg, V, s0, 1.0, lse, ent, dl, de, tp_dh, R, dW_shard=tp_dW, workspace=ws),
+        args.steps)
+    tp_line = {"tp": tp_world, "shard_rows": s1 - s0, "fwd_shard_ms": tp_f, "bwd_shard_ms": tp_b,
+               "tflops": 8.0 * T * H * (s1 - s0) / ((tp_f + tp_b) * 1e-3) / 1e12,
+               "note": "rank 0's kernels on one GPU; the all-gathers / all-to-all are not "
+                       "included"}
+    del tp_dh, tp_dW
 
     # ---------------------------------------------------------------- end to end, host buffers
     hid_h = torch.from_numpy(w.hidden.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -412,6 +488,9 @@ def run_ours(args):
                                 "vocab-row slices, then the rank-ordered sum (rlk_sum_ordered)",
                         "bytes_sent_per_rank": (int((world - 1) * -(-V // world) * H * 4)
                                                 if use_rs else 0)},
+        "decode_fwd": decode,
+        "tp_shard": dict(tp_line, frac=tp_line["tflops"] / pk["bf16_tflops"],
+                         peak=pk["bf16_tflops"]),
         "clocks": clk.summary(),
         "device_error_flags": flags,
     }

@@ -11,6 +11,7 @@
 #include <cuda_runtime.h>
 
 #include "rlk.h"
+#include "rlk_decode.cuh"
 #include "rlk_kernel.cuh"
 
 namespace rlk {
@@ -218,10 +219,84 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
 // vocab rows v0 .. v0 + Vloc) with the online epilogue, writing one triple per
 // (row, 512-column split) to part_* ([T][ceil(Vloc / 512)]) and, for rows whose
 // target falls in these rows, the target's scaled logit to ytgt.
+static_assert(kDecSplit == kBN * kFwdGroup, "both forward kernels must use the same splits");
+
+int g_dec_max_clusters[kDecMaxRows / 16][kMaxDevices];  // by N / 16 - 1
+
+// Forward partials for T <= kDecMaxRows (decode_fwd_kernel, rlk_decode.cuh).
+rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
+                                      const int64_t* targets, int64_t T, int64_t H, int64_t Vloc,
+                                      int64_t v0, float temperature, float* part_m, float* part_s,
+                                      float* part_b, int64_t ldp, float* ytgt, uint32_t* err,
+                                      cudaStream_t st) {
+  DecArgs a;
+  a.N = T <= 16 ? 16 : static_cast<int>(ceil_div(T, 32) * 32);
+  if (!map_kmajor(&a.w_k, W, H, Vloc, H, kBM) || !map_kmajor(&a.hid_k, hidden, H, T, H, a.N))
+    return RLK_ERR_CUDA;
+  a.ep.targets = targets;
+  a.ep.part_m = part_m;
+  a.ep.part_s = part_s;
+  a.ep.part_b = part_b;
+  a.ep.ytgt = ytgt;
+  a.ep.T = static_cast<int>(T);
+  a.ep.V = static_cast<int>(Vloc);
+  a.ep.ldp = static_cast<int>(ldp);
+  a.ep.v0 = v0;
+  a.ep.scale_log2 = kLog2e / temperature;
+  a.err = err;
+  a.KB = static_cast<int>(H / kBK);
+  a.NG = static_cast<int>(fwd_groups(Vloc));
+  constexpr uint32_t kSmemLimit = 227u * 1024u;
+  a.stages = kDecMaxStages;
+  while (a.stages > 2 && dec_smem_bytes(a.N, a.stages) > kSmemLimit) --a.stages;
+  const uint32_t smem = dec_smem_bytes(a.N, a.stages);
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(decode_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemLimit)) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kDecCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int& mc = g_dec_max_clusters[a.N / 16 - 1][dev];
+  if (mc == 0) {
+    cfg.gridDim = dim3(kDecCluster);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_fwd_kernel, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return RLK_ERR_CUDA;
+    }
+    mc = n;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(kDecCluster * std::min<int>(a.NG, mc)));
+  if (cudaLaunchKernelEx(&cfg, decode_fwd_kernel, a) != cudaSuccess) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  return RLK_OK;
+}
+
 rlk_status enqueue_fwd_partials(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
                                 int64_t T, int64_t H, int64_t Vloc, int64_t v0, float temperature,
                                 float* part_m, float* part_s, float* part_b, int64_t ldp,
                                 float* ytgt, uint32_t* err, cudaStream_t st) {
+  if (T <= kDecMaxRows)
+    return enqueue_fwd_partials_short(hidden, W, targets, T, H, Vloc, v0, temperature, part_m,
+                                      part_s, part_b, ldp, ytgt, err, st);
   FwdArgs a;
   if (!map_kmajor(&a.hid_k, hidden, H, T, H, kBM) || !map_kmajor(&a.w_k, W, H, Vloc, H, kBM))
     return RLK_ERR_CUDA;

@@ -38,6 +38,50 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 //   end_unit(p, st, g)              once per unit
 // =====================================================================
 
+// One 32-column chunk of the forward's online update for one row: columns
+// col0 .. col0+31 of this W, y = x * log2(e) / tau already formed with
+// fwd_scale.  Masks columns >= V, records y at the target's local column, then
+// moves m to the chunk's max, rescales s and b, and adds the chunk's terms in
+// column order.  Both forward kernels run exactly this code; the _rn
+// intrinsics keep the compiler from fusing a product into a later add
+// differently in the two.
+__device__ __forceinline__ float fwd_scale(float x, float scale_log2) {
+  return __fmul_rn(x, scale_log2);
+}
+
+__device__ __forceinline__ void fwd_chunk_update(float (&y)[32], int col0, int V, int64_t tgt,
+                                                 float* ytgt_row, float& m, float& s,
+                                                 float& b) {
+  if (col0 + 32 > V) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j >= V) y[j] = kMaskLogit;
+  }
+  const int64_t d = tgt - col0;
+  if (d >= 0 && d < 32) {
+    float yt = y[0];
+#pragma unroll
+    for (int j = 1; j < 32; ++j) yt = (j == d) ? y[j] : yt;
+    *ytgt_row = yt;
+  }
+  float cm = y[0];
+#pragma unroll
+  for (int j = 1; j < 32; ++j) cm = fmaxf(cm, y[j]);
+  const float mn = fmaxf(m, cm);
+  const float dm = __fsub_rn(m, mn);
+  const float a = ex2_approx(dm);
+  b = __fmul_rn(a, fmaf(dm, s, b));
+  s = __fmul_rn(s, a);
+  m = mn;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float dd = __fsub_rn(y[j], mn);
+    const float e = ex2_approx(dd);
+    s = __fadd_rn(s, e);
+    b = fmaf(e, dd, b);
+  }
+}
+
 // Forward: per row, over the unit's vocab tiles in ascending order, keep the
 // online triple in base-2 units of y = x * log2(e) / tau:
 //   m = max y,  s = sum 2^(y - m),  b = sum 2^(y - m) (y - m)
@@ -77,37 +121,10 @@ struct EpiFwd {
     for (int c = 0; c < kBN / 32; ++c) {
       uint32_t r[32];
       tmem_ld32(taddr + c * 32, r);
-      const int col0 = nt * kBN + c * 32;
       float y[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(r[j]) * p.scale_log2;
-      if (col0 + 32 > p.V) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col0 + j >= p.V) y[j] = kMaskLogit;
-      }
-      const int64_t d = st.tgt - col0;
-      if (d >= 0 && d < 32) {
-        float yt = y[0];
-#pragma unroll
-        for (int j = 1; j < 32; ++j) yt = (j == d) ? y[j] : yt;
-        p.ytgt[st.row] = yt;
-      }
-      float cm = y[0];
-#pragma unroll
-      for (int j = 1; j < 32; ++j) cm = fmaxf(cm, y[j]);
-      const float mn = fmaxf(st.m, cm);
-      const float a = ex2_approx(st.m - mn);
-      st.b = a * fmaf(st.m - mn, st.s, st.b);
-      st.s = st.s * a;
-      st.m = mn;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float dd = y[j] - mn;
-        const float e = ex2_approx(dd);
-        st.s += e;
-        st.b = fmaf(e, dd, st.b);
-      }
+      for (int j = 0; j < 32; ++j) y[j] = fwd_scale(__uint_as_float(r[j]), p.scale_log2);
+      fwd_chunk_update(y, nt * kBN + c * 32, p.V, st.tgt, p.ytgt + st.row, st.m, st.s, st.b);
     }
   }
 
