@@ -200,3 +200,39 @@ def sweep_batch(T: int, probes, filler_seed: int, H: int = QWEN_H, V: int = QWEN
     dlogp[pos] = pdl[:n]
     dent[pos] = pde[:n]
     return hidden, targets, dlogp, dent, probe_idx, pos
+
+
+# --------------------------------------------------------------------------
+# Diffusion transition step (the RL-Kernel B200 report's transition gate,
+# h3-runtime-integration-b200 report.json, transition[].shape): B samples of
+# L x D latent elements.
+TRANSITION_SHAPES = ((3, 257 * 96), (4, 4096 * 96), (2, 8192 * 32))   # (B, n = L * D)
+
+
+@dataclasses.dataclass
+class TransitionCase:
+    B: int
+    n: int
+    x: np.ndarray    # [B, n] float32 latent
+    v: np.ndarray    # [B, n] float32 model output
+    eps: np.ndarray  # [B, n] float32 standard normal draw for sampling
+    a: np.ndarray    # [B] float32 per-sample coefficient of x
+    c: np.ndarray    # [B] float32 per-sample coefficient of v
+    s: np.ndarray    # [B] float32 per-sample transition std (> 0)
+
+
+def transition_case(seed: int, B: int, n: int) -> TransitionCase:
+    """Seeded float32 inputs: x, v, eps ~ N(0, 1); a ~ U(0.98, 1.02) (a step
+    close to the identity), c ~ U(-0.1, -0.01) (a small step along the model
+    output), s ~ U(0.05, 0.5)."""
+    ss = np.random.SeedSequence([seed, B, n, 0x7A51])
+    r = [np.random.default_rng(k) for k in ss.spawn(6)]
+    f32 = np.float32
+    return TransitionCase(
+        B, n,
+        r[0].standard_normal((B, n)).astype(f32),
+        r[1].standard_normal((B, n)).astype(f32),
+        r[2].standard_normal((B, n)).astype(f32),
+        r[3].uniform(0.98, 1.02, B).astype(f32),
+        r[4].uniform(-0.1, -0.01, B).astype(f32),
+        r[5].uniform(0.05, 0.5, B).astype(f32))

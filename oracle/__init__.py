@@ -6,7 +6,9 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 
 ``rlk_oracle.c`` is the oracle proper (plain C, OpenMP over rows/vocab, fp64,
 two-pass softmax); ``brute.py`` is an independent dense numpy float64 brute
-force used to pin it on tiny inputs.  See the header of ``rlk_oracle.c`` for
+force used to pin it on tiny inputs.  ``transition.py`` is the fp64 numpy
+oracle of the diffusion transition step (pinned by
+tests/test_transition_oracle.py).  See the header of ``rlk_oracle.c`` for
 the definition each step follows and the passages it rests on.
 
 Pinned by tests/test_oracle_pins.py: brute force on tiny inputs, the uniform
