@@ -328,6 +328,43 @@ def run_ours(args):
               "eager_us_per_call": [e for _, e in dec_us], "achieved": dec_gbs,
               "frac": [g / peaks()[0]["hbm_gbs"] for g in dec_gbs]}
 
+    # ---------------------------------------------------------------- diffusion transition step
+    # The report's three transition shapes; one sampling step (reads x, v,
+    # eps; writes mean, prev_sample, logp: 20 bytes per element).  A sampler
+    # loop captured whole: 20 steps in one CUDA graph, replayed 10 times.  At
+    # these sizes (1.5-31 MB per step) launch gaps still set much of the time.
+    from invariant_lm_head_gemm_b200 import workloads as wlm
+    trans = {"kernel": "transition_kernel (one launch per step)", "bound": "hbm",
+             "unit": "GB/s", "timing": "CUDA graph of 20 steps, replayed 10 times", "shapes": [],
+             "us_per_call": [], "achieved": [], "frac": []}
+    for i, (Bt, nt) in enumerate(wlm.TRANSITION_SHAPES):
+        tw = wlm.transition_case(i, Bt, nt)
+        tx, tv, te, ta, tc, tsd = (torch.from_numpy(np.ascontiguousarray(q)).to(dev)
+                                   for q in (tw.x, tw.v, tw.eps, tw.a, tw.c, tw.s))
+        t_ws = binding.transition_workspace(Bt, nt, dev)
+        t_out = (torch.empty_like(tx), torch.empty_like(tx), torch.empty(Bt, device=dev))
+        binding.rlk_transition_sample(tx, tv, te, ta, tc, tsd, out=t_out, workspace=t_ws)
+        tg_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tg_graph):
+            for _ in range(20):
+                binding.rlk_transition_sample(tx, tv, te, ta, tc, tsd, out=t_out, workspace=t_ws)
+        for _ in range(2):
+            tg_graph.replay()
+        ta0 = torch.cuda.Event(enable_timing=True)
+        ta1 = torch.cuda.Event(enable_timing=True)
+        ta0.record(stream)
+        for _ in range(10):
+            tg_graph.replay()
+        ta1.record(stream)
+        torch.cuda.synchronize()
+        t_us = 1e3 * ta0.elapsed_time(ta1) / 200
+        t_gbs = (20 * Bt * nt + 16 * Bt) / (t_us * 1e-6) / 1e9
+        trans["shapes"].append([Bt, nt])
+        trans["us_per_call"].append(t_us)
+        trans["achieved"].append(t_gbs)
+        trans["frac"].append(t_gbs / peaks()[0]["hbm_gbs"])
+        del tg_graph
+
     # ---------------------------------------------------------------- device-resident
     for _ in range(args.warmup):
         step()
@@ -489,6 +526,7 @@ def run_ours(args):
                         "bytes_sent_per_rank": (int((world - 1) * -(-V // world) * H * 4)
                                                 if use_rs else 0)},
         "decode_fwd": decode,
+        "transition": trans,
         "tp_shard": dict(tp_line, frac=tp_line["tflops"] / pk["bf16_tflops"],
                          peak=pk["bf16_tflops"]),
         "clocks": clk.summary(),

@@ -82,6 +82,7 @@ typedef enum {
 /* Bits of the device error word at the start of the workspace. */
 #define RLK_DEVERR_TARGET 0x1u
 #define RLK_DEVERR_TIMEOUT 0x2u
+#define RLK_DEVERR_SCALE 0x4u   /* a transition std s_b was not a positive finite number */
 
 /* Bytes of workspace that rlk_linear_logp_fwd (for_backward == 0) or both
  * rlk_linear_logp_fwd and rlk_linear_logp_bwd (for_backward != 0) need for
@@ -223,6 +224,44 @@ rlk_status rlk_linear_logp_bwd_shard(const rlk_bf16* hidden, const rlk_bf16* W_s
                                      size_t workspace_bytes, void* stream);
 rlk_status rlk_dhidden_combine(const float* dh_parts, int64_t nparts, int64_t count,
                                rlk_bf16* out, void* stream);
+
+/* Diffusion transition step and its log-probability.  The RL-Kernel B200
+ * report's transition gate (h3-runtime-integration-b200 report.json,
+ * transition[]: shapes B3 x 257x96, B4 x 4096x96, B2 x 8192x32; prev_sample and
+ * mean bitwise, logp within 5.8e-6 .. 1.5e-4 of a torch mean, batch invariant,
+ * scoring reproduces the sampling logprob) checks such an operator but gives
+ * no formula; this library takes the plainest reading, a Gaussian transition
+ * with an affine mean, per sample b of n = L * D elements:
+ *     mean = a_b x + c_b v,   prev = mean + s_b eps,
+ *     logp_b = mean over the n elements of log N(prev; mean, s_b^2)
+ *            = -(sum (prev - mean)^2) / (2 s_b^2 n) - ln s_b - ln(2 pi) / 2.
+ * x (latent), v (model output), eps (standard normal draw), prev: fp32
+ * [B][n] row-major, 16-byte aligned; a, c, s: fp32 [B]; mean_out (may be
+ * NULL) and prev_out fp32 [B][n], 16-byte aligned; logp fp32 [B].
+ * Elementwise results are single fp32 operations rounded to nearest (a x,
+ * c v, their sum; s eps, mean + that), so mean and prev equal plain fp32
+ * tensor arithmetic bit for bit.  The residual sum of a sample runs over fixed
+ * 4096-element chunks in a fixed order and then over the chunks in order:
+ * logp is bitwise independent of B and of the other samples, and
+ * rlk_transition_logp on a recorded prev reproduces rlk_transition_sample's
+ * logp bit for bit.
+ * Sizes: n % 4 == 0, n <= 2^24, B <= 65535 (else RLK_ERR_UNSUPPORTED_SHAPE);
+ * B = 0 or n = 0 is a no-op.  Workspace: rlk_transition_workspace_bytes(B, n)
+ * bytes, 256-byte aligned, caller-owned, ZERO-FILLED ONCE before its first use
+ * (every call leaves its counters at zero again; calls sharing a workspace
+ * must not overlap on the GPU).  Its first word is the device error word,
+ * rewritten by every call: a non-positive or non-finite s_b gives NaN logp_b
+ * and sets RLK_DEVERR_SCALE.  One kernel is enqueued on `stream`; nothing is
+ * allocated. */
+size_t rlk_transition_workspace_bytes(int64_t B, int64_t n);
+rlk_status rlk_transition_sample(const float* x, const float* v, const float* eps,
+                                 const float* a, const float* c, const float* s, int64_t B,
+                                 int64_t n, float* mean_out, float* prev_out, float* logp,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+rlk_status rlk_transition_logp(const float* x, const float* v, const float* prev,
+                               const float* a, const float* c, const float* s, int64_t B,
+                               int64_t n, float* mean_out, float* logp, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /* Batch-invariant deterministic dense GEMM on the same tensor-core mainloop as
  * every kernel above (also its self-check): C[M,N] fp32 = sum_k A[m,k] B[n,k]

@@ -383,3 +383,77 @@ def rlk_dhidden_combine(dh_parts, nparts, out, stream=None):
     _check(_tp().rlk_dhidden_combine(_ptr(dh_parts), nparts, count, _ptr(out), _stream(stream)),
            "rlk_dhidden_combine")
     return out
+
+
+_tr_fns = None
+
+
+def _tr():
+    global _tr_fns
+    if _tr_fns is None:
+        L = lib()
+        L.rlk_transition_workspace_bytes.argtypes = [_I64, _I64]
+        L.rlk_transition_workspace_bytes.restype = ctypes.c_size_t
+        L.rlk_transition_sample.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P,
+                                            ctypes.c_size_t, _P]
+        L.rlk_transition_sample.restype = ctypes.c_int
+        L.rlk_transition_logp.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P,
+                                          ctypes.c_size_t, _P]
+        L.rlk_transition_logp.restype = ctypes.c_int
+        _tr_fns = L
+    return _tr_fns
+
+
+def transition_workspace(B: int, n: int, device=None):
+    nbytes = _tr().rlk_transition_workspace_bytes(B, n)
+    if nbytes == 0:
+        raise ValueError("unsupported sizes B=%d n=%d" % (B, n))
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def _tr_args(x, v, third, a, c, s):
+    for t, name in ((x, "x"), (v, "v"), (third, "eps/prev")):
+        _req(t, torch.float32, name, 2)
+    for t, name in ((a, "a"), (c, "c"), (s, "s")):
+        _req(t, torch.float32, name, 1)
+    B, n = x.shape
+    if v.shape != x.shape or third.shape != x.shape or a.shape[0] != B or c.shape[0] != B \
+            or s.shape[0] != B:
+        raise ValueError("x, v, eps/prev must be [B, n]; a, c, s [B]")
+    return B, n
+
+
+def rlk_transition_sample(x, v, eps, a, c, s, want_mean=True, out=None, workspace=None,
+                          stream=None):
+    """(mean or None, prev, logp) of one sampling step: x, v, eps fp32 [B, n]
+    (n = L * D flattened), a, c, s fp32 [B]."""
+    B, n = _tr_args(x, v, eps, a, c, s)
+    if out is None:
+        out = (torch.empty_like(x) if want_mean else None, torch.empty_like(x),
+               torch.empty(B, dtype=torch.float32, device=x.device))
+    mean, prev, logp = out
+    if workspace is None:
+        workspace = transition_workspace(B, n, x.device)
+    _check(_tr().rlk_transition_sample(_ptr(x), _ptr(v), _ptr(eps), _ptr(a), _ptr(c), _ptr(s), B,
+                                       n, _ptr(mean) if mean is not None else None, _ptr(prev),
+                                       _ptr(logp), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)),
+           "rlk_transition_sample")
+    return mean, prev, logp
+
+
+def rlk_transition_logp(x, v, prev, a, c, s, want_mean=False, out=None, workspace=None,
+                        stream=None):
+    """(mean or None, logp) of scoring a recorded prev_sample."""
+    B, n = _tr_args(x, v, prev, a, c, s)
+    if out is None:
+        out = (torch.empty_like(x) if want_mean else None,
+               torch.empty(B, dtype=torch.float32, device=x.device))
+    mean, logp = out
+    if workspace is None:
+        workspace = transition_workspace(B, n, x.device)
+    _check(_tr().rlk_transition_logp(_ptr(x), _ptr(v), _ptr(prev), _ptr(a), _ptr(c), _ptr(s), B,
+                                     n, _ptr(mean) if mean is not None else None, _ptr(logp),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+           "rlk_transition_logp")
+    return mean, logp

@@ -12,6 +12,7 @@
 
 #include "rlk.h"
 #include "rlk_decode.cuh"
+#include "rlk_device.h"
 #include "rlk_kernel.cuh"
 
 namespace rlk {
@@ -404,6 +405,9 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
 }
 
 }  // namespace
+
+rlk_status current_device_supported(int* num_sms) { return check_device(num_sms); }
+
 }  // namespace rlk
 
 using namespace rlk;

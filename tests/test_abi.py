@@ -125,6 +125,9 @@ def test_valid_call_without_a_gpu_is_refused(L):
     assert L.rlk_gemm_bf16_f32(A16, A16, 8, 8, 8, 0, 0, A16, A256, 256, None) == DEVICE
     assert _shard(L) == DEVICE and _combine(L) == DEVICE
     assert _bshard(L) == DEVICE and L.rlk_dhidden_combine(A16, 2, 8, A16, None) == DEVICE
+    binding._tr()
+    assert L.rlk_transition_sample(A16, A16, A16, A16, A16, A16, 2, 8, None, A16, A16, A256,
+                                   1 << 20, None) == DEVICE
     assert binding.call_count(0) == 0 and binding.call_count(1) == 0
 
 
@@ -199,3 +202,28 @@ def test_tp_backward_argument_errors(L):
     assert c(None, 2, 8, A16, None) == INVALID
     assert c(A16 + 4, 2, 8, A16, None) == MISALIGNED
     assert c(A16, 2, 8, A16 + 2, None) == MISALIGNED
+
+
+def test_transition_argument_errors(L):
+    binding._tr()
+    S = L.rlk_transition_sample
+    need = L.rlk_transition_workspace_bytes(3, 24672)
+    assert need > 256 and L.rlk_transition_workspace_bytes(-1, 4) == 0
+
+    def smp(B=3, n=24672, x=A16, prev=A16, ws=A256, wsb=need, mean=A16):
+        return S(x, A16, A16, A16, A16, A16, B, n, mean, prev, A16, ws, wsb, None)
+
+    assert smp(n=6) == SHAPE                  # n % 4
+    assert smp(B=70000) == SHAPE
+    assert smp(n=(1 << 24) + 4) == SHAPE
+    assert smp(B=-1) == INVALID
+    assert smp(B=0, x=None) == OK             # empty: no-op
+    assert smp(x=None) == INVALID
+    assert smp(prev=None) == INVALID          # sampling writes prev
+    assert smp(mean=None) != INVALID          # the mean output is optional
+    assert smp(x=A16 + 4) == MISALIGNED
+    assert smp(ws=A256 + 16) == MISALIGNED
+    assert smp(wsb=need - 1) == WS_SMALL
+    lg = L.rlk_transition_logp
+    assert lg(A16, A16, None, A16, A16, A16, 3, 24672, None, A16, A256, need, None) == INVALID
+    assert lg(A16, A16, A16, A16, A16, A16, 3, 10, None, A16, A256, need, None) == SHAPE
