@@ -373,11 +373,13 @@ def run_ours(args):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        torch.cuda.nvtx.range_push("rl_step_timed")   # lets ncu capture just this region
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max, tokens_all = aggregate(ms, T)
@@ -544,6 +546,19 @@ def run_profile(args):
     from invariant_lm_head_gemm_b200 import binding
     from invariant_lm_head_gemm_b200 import workloads as wl
 
+    if args.profile == "transition":
+        B, n = wl.TRANSITION_SHAPES[1]
+        tw = wl.transition_case(1, B, n)
+        dev = torch.device("cuda", 0)
+        tx, tv, te, ta, tc, ts = (torch.from_numpy(np.ascontiguousarray(q)).to(dev)
+                                  for q in (tw.x, tw.v, tw.eps, tw.a, tw.c, tw.s))
+        ws = binding.transition_workspace(B, n, dev)
+        for _ in range(args.iters):
+            binding.rlk_transition_sample(tx, tv, te, ta, tc, ts, workspace=ws)
+        torch.cuda.synchronize()
+        print("profile case done: transition B=%d n=%d iters=%d flags=%d" % (
+            B, n, args.iters, binding.rlk_read_device_error(ws)))
+        return 0
     T, H, V = args.T, 4096, args.V
     hidden, targets = wl.make_rows(5, T, H, V)
     W = wl.make_weight(5, V, H)
@@ -578,7 +593,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=2)
     ap.add_argument("--no-dw-reduce", action="store_true",
                     help="N > 1: leave out the deterministic dW reduce-scatter from the step")
-    ap.add_argument("--profile", choices=["fwd", "bwd"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "bwd", "transition"], default=None,
                     help="run a small case for an ncu capture instead of the benchmark")
     ap.add_argument("--T", type=int, default=2048, help="rows of the --profile case")
     ap.add_argument("--V", type=int, default=32768, help="vocab of the --profile case")

@@ -82,14 +82,24 @@ __global__ void __launch_bounds__(kTrThreads) transition_kernel(
   // squared residuals: per thread over its float4s in order, x+y and z+w
   // first; then a warp butterfly (every lane ends with the same sum); then
   // the warps in order
-  float acc = 0.f;
+  // every load of the thread is issued before any arithmetic: the kernel is
+  // one DRAM round trip deep
+  float4 xs[kTrVecs], vs[kTrVecs], ts[kTrVecs];
 #pragma unroll
   for (int k = 0; k < kTrVecs; ++k) {
     const int64_t i = c0 + (static_cast<int64_t>(k) * kTrThreads + threadIdx.x) * 4;
     if (i < n) {  // n % 4 == 0: the whole float4 is inside the sample
-      const float4 xv = *reinterpret_cast<const float4*>(x + base + i);
-      const float4 vv = *reinterpret_cast<const float4*>(v + base + i);
-      const float4 tv = *reinterpret_cast<const float4*>(third + base + i);
+      xs[k] = __ldcs(reinterpret_cast<const float4*>(x + base + i));
+      vs[k] = __ldcs(reinterpret_cast<const float4*>(v + base + i));
+      ts[k] = __ldcs(reinterpret_cast<const float4*>(third + base + i));
+    }
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < kTrVecs; ++k) {
+    const int64_t i = c0 + (static_cast<int64_t>(k) * kTrThreads + threadIdx.x) * 4;
+    if (i < n) {
+      const float4 xv = xs[k], vv = vs[k], tv = ts[k];
       const float4 mu = mean4(ab, xv, cb, vv);
       float4 pr = tv;
       if constexpr (kSample) {
