@@ -152,6 +152,24 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// MN-major operand stored [K, MN] (MN contiguous, pitch elements per K row)
+// mapped 3-D as (64 MN, K, MN / 64) with box 64 x 64 x 2: one copy lands the
+// 128 MN columns of a stage as two 8 KB 64 x 64 swizzled blocks back to back,
+// the same bytes and layout as two 2-D boxes.  Needs MN % 64 == 0; false if
+// the driver declines the map.
+bool map_mnmajor3(CUtensorMap* m, const void* base, int64_t MN, int64_t K, int64_t pitch) {
+  if (MN % 64 != 0) return false;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(MN / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(pitch) * 2, 128};
+  cuuint32_t box[3] = {64, 64, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // K-major operand [rows, K] (K contiguous): one 64 x box_rows box per stage.
 bool map_kmajor(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t pitch,
                 uint32_t box_rows) {
@@ -363,16 +381,27 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   P.plan = make_bwd_plan(T, H, Vloc, vchunk(Vfull));
   const BwdPlan& pl = P.plan;
   if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
-      !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM) || !map_mnmajor(&P.maps.w_mn, W, H, Vloc, H) ||
-      !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
+      !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM))
     return RLK_ERR_CUDA;
   for (int i = 0; i < kDxBuffers; ++i) {
     P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
     if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx) ||
         !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
       return RLK_ERR_CUDA;
   }
+  // MN-major operands of the dHidden and dW units: 3-D maps (half the copies)
+  // when the driver takes them, else 2-D maps; same shared-memory bytes.
+  bool mn3 = map_mnmajor3(&P.maps.w_mn, W, H, Vloc, H) &&
+             map_mnmajor3(&P.maps.hid_mn, hidden, H, T, H);
+  for (int i = 0; mn3 && i < kDxBuffers; ++i)
+    mn3 = map_mnmajor3(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx);
+  if (!mn3) {
+    if (!map_mnmajor(&P.maps.w_mn, W, H, Vloc, H) || !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
+      return RLK_ERR_CUDA;
+    for (int i = 0; i < kDxBuffers; ++i)
+      if (!map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx)) return RLK_ERR_CUDA;
+  }
+  P.mn3 = mn3 ? 1 : 0;
   P.targets = targets;
   P.lse = lse;
   P.entropy = entropy;
@@ -503,8 +532,11 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
   uint32_t* err = static_cast<uint32_t*>(workspace);
 
   GemmArgs a;
-  bool ok = a_mn_major ? map_mnmajor(&a.a, A, M, K, M) : map_kmajor(&a.a, A, K, M, K, kBM);
-  ok = ok && (b_mn_major ? map_mnmajor(&a.b, B, N, K, N) : map_kmajor(&a.b, B, K, N, K, kBM));
+  a.a3 = a_mn_major && map_mnmajor3(&a.a, A, M, K, M) ? 1 : 0;
+  a.b3 = b_mn_major && map_mnmajor3(&a.b, B, N, K, N) ? 1 : 0;
+  bool ok = a.a3 || (a_mn_major ? map_mnmajor(&a.a, A, M, K, M) : map_kmajor(&a.a, A, K, M, K, kBM));
+  ok = ok && (a.b3 || (b_mn_major ? map_mnmajor(&a.b, B, N, K, N)
+                                  : map_kmajor(&a.b, B, K, N, K, kBM)));
   if (!ok) return RLK_ERR_CUDA;
   a.ep.out = C;
   a.ep.rows = static_cast<int>(M);

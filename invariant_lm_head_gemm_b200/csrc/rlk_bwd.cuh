@@ -38,10 +38,10 @@ constexpr int kDxBuffers = 3;
 struct BwdMaps {
   CUtensorMap hid_k;              // hidden [T,H], K-major, box 64 x 128
   CUtensorMap w_k;                // W [V,H], K-major, box 64 x 256
-  CUtensorMap w_mn;               // W read as MN-major (N = h, K = v), box 64 x 64
-  CUtensorMap hid_mn;             // hidden read as MN-major (N = h, K = t), box 64 x 64
+  CUtensorMap w_mn;               // W read as MN-major (N = h, K = v), box 64 x 64 (x 2 when 3-D)
+  CUtensorMap hid_mn;             // hidden read as MN-major (N = h, K = t), box 64 x 64 (x 2)
   CUtensorMap dx_k[kDxBuffers];   // dX buffer [T, ldx], K-major, box 64 x 128
-  CUtensorMap dx_mn[kDxBuffers];  // dX buffer read as MN-major (M = v, K = t), box 64 x 64
+  CUtensorMap dx_mn[kDxBuffers];  // dX buffer read as MN-major (M = v, K = t), box 64 x 64 (x 2)
   CUtensorMap dx_st[kDxBuffers];  // dX buffer written by TMA stores, box 32 x 32, no swizzle
 };
 
@@ -80,6 +80,7 @@ struct BwdParams {
   uint32_t* err;
   float scale_log2;   // log2(e) / tau
   float inv_tau;
+  int mn3;            // w_mn, hid_mn, dx_mn are 3-D maps (one box per 128 MN columns)
 };
 
 enum : int { kUnitR = 0, kUnitH = 1, kUnitD = 2 };

@@ -55,12 +55,13 @@ struct FwdArgs {
 };
 
 struct GemmArgs {
-  CUtensorMap a;      // K-major box 64 x 128, or MN-major box 64 x 64
+  CUtensorMap a;      // K-major box 64 x 128, or MN-major box 64 x 64 (64 x 64 x 2 when a3)
   CUtensorMap b;
   EpiStore::Params ep;
   uint32_t* err;
   int M, N, MT, NT, KB;
   int a_mn, b_mn;
+  int a3, b3;
   long long total;
 };
 
@@ -88,6 +89,7 @@ struct Job {
   int ntiles;       // N tiles in the unit
   int kbs;          // K blocks per tile
   bool a_mn, b_mn;  // operand majorness
+  bool a3, b3;      // MN-major operand mapped 3-D: one box per 128 MN columns (else two 2-D boxes)
   const CUtensorMap* mA;
   const CUtensorMap* mB;
   int a_row0;       // M coordinate of the tile's first row in A's tensor map
@@ -107,6 +109,7 @@ __device__ __forceinline__ Job make_job(const FwdArgs& P, long long u) {
   j.ntiles = min(P.group, P.NT - j.nt);
   j.kbs = P.KB;
   j.a_mn = j.b_mn = false;
+  j.a3 = j.b3 = false;
   j.mA = &P.hid_k;
   j.mB = &P.w_k;
   j.a_row0 = j.mt * kPairM;
@@ -127,6 +130,8 @@ __device__ __forceinline__ Job make_job(const GemmArgs& P, long long u) {
   j.kbs = P.KB;
   j.a_mn = P.a_mn != 0;
   j.b_mn = P.b_mn != 0;
+  j.a3 = P.a3 != 0;
+  j.b3 = P.b3 != 0;
   j.mA = &P.a;
   j.mB = &P.b;
   j.a_row0 = j.mt * kPairM;
@@ -147,6 +152,7 @@ __device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
   j.nt = un.b;
   j.ntiles = 1;
   j.bk0 = 0;
+  j.a3 = j.b3 = false;
   const int buf = un.c % kDxBuffers;
   if (un.type == kUnitR) {
     j.kbs = pl.KB_R;
@@ -163,6 +169,7 @@ __device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
     j.b_mn = true;
     j.mA = &P.maps.dx_k[buf];
     j.mB = &P.maps.w_mn;
+    j.b3 = P.mn3 != 0;
     j.a_row0 = un.a * kPairM;
     j.b_col0 = un.b * kBN;
     j.bk0 = un.c * pl.ldx;
@@ -173,6 +180,7 @@ __device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
     j.a_mn = j.b_mn = true;
     j.mA = &P.maps.dx_mn[buf];
     j.mB = &P.maps.hid_mn;
+    j.a3 = j.b3 = P.mn3 != 0;
     j.a_row0 = un.a * kPairM;
     j.b_col0 = un.b * kBN;
     j.a_ext = pl.ldx;
@@ -194,6 +202,8 @@ __device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank
   const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
   if (!j.a_mn) {
     if (a0 < j.a_ext) bytes += kPAStage;
+  } else if (j.a3) {
+    if (a0 < j.a_ext) bytes += 2 * kBox;  // the box counts in full, past-the-end half filled
   } else {
     if (a0 < j.a_ext) bytes += kBox;
     if (a0 + 64 < j.a_ext) bytes += kBox;
@@ -201,6 +211,8 @@ __device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank
   const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
   if (!j.b_mn) {
     if (b0 < j.b_ext) bytes += kPBStage;
+  } else if (j.b3) {
+    if (b0 < j.b_ext) bytes += 2 * kBox;
   } else {
     if (b0 < j.b_ext) bytes += kBox;
     if (b0 + 64 < j.b_ext) bytes += kBox;
@@ -351,12 +363,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int k = kb * kBK;
             if (!j.a_mn) {
               if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, k, a0);
+            } else if (j.a3) {
+              if (a0 < j.a_ext) tma_load_3d_pair(dA, j.mA, fb, 0, k, a0 >> 6);
             } else {
               if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, a0, k);
               if (a0 + 64 < j.a_ext) tma_load_2d_pair(dA + kBox, j.mA, fb, a0 + 64, k);
             }
             if (!j.b_mn) {
               if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, k, b0);
+            } else if (j.b3) {
+              if (b0 < j.b_ext) tma_load_3d_pair(dB, j.mB, fb, 0, j.bk0 + k, b0 >> 6);
             } else {
               if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, b0, j.bk0 + k);
               if (b0 + 64 < j.b_ext) tma_load_2d_pair(dB + kBox, j.mB, fb, b0 + 64, j.bk0 + k);
