@@ -502,9 +502,8 @@ def run_ours(args):
     step_tflops = flops_tok * tokens_all / world / (ms_max * 1e-3) / 1e12
     fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = 6.0 * T * H * V / (bwd_ms * 1e-3) / 1e12
-    launches_per_step = 4 + (1 if use_rs else 0)   # fwd pair kernel, combine, hidden
-                                                    # transpose, bwd pair kernel (+ the
-                                                    # ordered sum of dW)
+    launches_per_step = 3 + (1 if use_rs else 0)   # fwd pair kernel, combine, bwd pair
+                                                    # kernel (+ the ordered sum of dW)
     value = tokens_all / (ms_max * 1e-3)
     line = {
         "metric": METRIC,

@@ -52,12 +52,8 @@ size_t bwd_counter_words(const BwdPlan& p) {
 
 struct Layout {
   size_t pm, ps, pb, yt, fwd_end;
-  size_t dx[kDxBuffers], dh, dxt[kDxBuffers], hidt, cnt, bwd_end;
+  size_t dx[kDxBuffers], dh, cnt, bwd_end;
 };
-
-// Row pitch (elements) of the transposed buffers [.., T]: T rounded up to 64,
-// so that every row starts on a 128-byte boundary.
-int64_t t_pitch(int64_t T) { return ceil_div(std::max<int64_t>(T, 1), 64) * 64; }
 
 Layout layout(int64_t T, int64_t H, int64_t V) {
   Layout L;
@@ -72,12 +68,7 @@ Layout layout(int64_t T, int64_t H, int64_t V) {
   L.dx[0] = kHeader;
   for (int i = 1; i < kDxBuffers; ++i) L.dx[i] = L.dx[i - 1] + dx_bytes;
   L.dh = L.dx[kDxBuffers - 1] + dx_bytes;
-  const size_t tp = static_cast<size_t>(t_pitch(T));
-  const size_t dxt_bytes = align256(static_cast<size_t>(vchunk(V)) * tp * 2);
-  L.dxt[0] = L.dh + align256(t * static_cast<size_t>(H) * 4);
-  for (int i = 1; i < kDxBuffers; ++i) L.dxt[i] = L.dxt[i - 1] + dxt_bytes;
-  L.hidt = L.dxt[kDxBuffers - 1] + dxt_bytes;
-  L.cnt = L.hidt + align256(static_cast<size_t>(H) * tp * 2);
+  L.cnt = L.dh + align256(t * static_cast<size_t>(H) * 4);
   L.bwd_end = L.cnt + align256(bwd_counter_words(bwd_plan(T, H, V)) * 4);
   return L;
 }
@@ -376,28 +367,6 @@ rlk_status enqueue_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
                          st);
 }
 
-// out[h][t] = in[t][h] for t < T (out rows have pitch ld >= T): hidden
-// transposed for the dW units' K-major B operand.  32 x 32 tiles through
-// shared memory (padded rows), coalesced on both sides.
-__global__ void __launch_bounds__(256) transpose_rows_kernel(const __nv_bfloat16* __restrict__ in,
-                                                             int T, int H,
-                                                             __nv_bfloat16* __restrict__ out,
-                                                             int ld) {
-  __shared__ uint16_t tile[32][33];
-  const int h0 = blockIdx.x * 32, t0 = blockIdx.y * 32;
-  const uint16_t* src = reinterpret_cast<const uint16_t*>(in);
-  uint16_t* dst = reinterpret_cast<uint16_t*>(out);
-  for (int r = threadIdx.y; r < 32; r += 8) {
-    const int t = t0 + r;
-    if (t < T) tile[r][threadIdx.x] = src[static_cast<size_t>(t) * H + h0 + threadIdx.x];
-  }
-  __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += 8) {
-    const int t = t0 + threadIdx.x;
-    if (t < T) dst[static_cast<size_t>(h0 + r) * ld + t] = tile[threadIdx.x][r];
-  }
-}
-
 // Backward over W rows [v0, v0 + Vloc) of a Vfull-row head (the whole head:
 // v0 = 0, Vloc = Vfull), chunked as the full head is.  dh_parts null: dHidden
 // accumulated over the chunks and written as bf16; else each chunk's fp32
@@ -414,22 +383,24 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
       !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM))
     return RLK_ERR_CUDA;
-  const int64_t tp = t_pitch(T);
   for (int i = 0; i < kDxBuffers; ++i) {
     P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
-    void* dxt = ws + L.dxt[i];
     if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !map_kmajor(&P.maps.dxt_k[i], dxt, T, pl.ldx, tp, kBM) ||
-        !make_map(&P.maps.dxt_st[i], dxt, T, pl.ldx, tp, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
       return RLK_ERR_CUDA;
   }
-  __nv_bfloat16* hidt = reinterpret_cast<__nv_bfloat16*>(ws + L.hidt);
-  if (!map_kmajor(&P.maps.hidt_k, hidt, T, H, tp, kBM)) return RLK_ERR_CUDA;
-  // W as the dHidden units' MN-major operand: a 3-D map (one copy per stage)
-  // when the driver takes it, else a 2-D map (two); same shared-memory bytes.
-  const bool mn3 = map_mnmajor3(&P.maps.w_mn, W, H, Vloc, H);
-  if (!mn3 && !map_mnmajor(&P.maps.w_mn, W, H, Vloc, H)) return RLK_ERR_CUDA;
+  // MN-major operands of the dHidden and dW units: 3-D maps (half the copies)
+  // when the driver takes them, else 2-D maps; same shared-memory bytes.
+  bool mn3 = map_mnmajor3(&P.maps.w_mn, W, H, Vloc, H) &&
+             map_mnmajor3(&P.maps.hid_mn, hidden, H, T, H);
+  for (int i = 0; mn3 && i < kDxBuffers; ++i)
+    mn3 = map_mnmajor3(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx);
+  if (!mn3) {
+    if (!map_mnmajor(&P.maps.w_mn, W, H, Vloc, H) || !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
+      return RLK_ERR_CUDA;
+    for (int i = 0; i < kDxBuffers; ++i)
+      if (!map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx)) return RLK_ERR_CUDA;
+  }
   P.mn3 = mn3 ? 1 : 0;
   P.targets = targets;
   P.lse = lse;
@@ -456,11 +427,6 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   P.inv_tau = 1.0f / temperature;
 
   if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
-  transpose_rows_kernel<<<dim3(static_cast<unsigned>(H / 32), static_cast<unsigned>(ceil_div(T, 32))),
-                          dim3(32, 8), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(hidden),
-                                                static_cast<int>(T), static_cast<int>(H), hidt,
-                                                static_cast<int>(tp));
-  if (cudaGetLastError() != cudaSuccess) return RLK_ERR_CUDA;
   // Units wait on units claimed earlier, and only running CTA pairs claim
   // units, so no pair ever waits on one that has not started: the launch needs
   // no co-residency guarantee.

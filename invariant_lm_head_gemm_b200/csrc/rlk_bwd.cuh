@@ -8,8 +8,7 @@
 //               (K = the chunk's vocab entries), chunks added in ascending
 //               order (old + new), the last one written as bf16;
 //   D(c, v, n)  dW[chunk c rows v, n cols] = dX_c[:, v]^T . hidden[:, n]
-//               (K = T, ascending, no atomics), read K-major from the
-//               transposed copies the R units and a transpose kernel write.
+//               (K = T, ascending, no atomics).
 // Global order: R(0), R(1), then for g = 0 .. NC-1: H(g), D(g), R(g + 2).
 // Every dependency points to an earlier unit, one group back or more:
 //   H(c, m, .) needs every R(c, m, .)            (counter rdone_m[c][m])
@@ -40,11 +39,10 @@ struct BwdMaps {
   CUtensorMap hid_k;              // hidden [T,H], K-major, box 64 x 128
   CUtensorMap w_k;                // W [V,H], K-major, box 64 x 256
   CUtensorMap w_mn;               // W read as MN-major (N = h, K = v), box 64 x 64 (x 2 when 3-D)
-  CUtensorMap hidt_k;             // hiddenT [H, Tp] (K = t), K-major, box 64 x 128
+  CUtensorMap hid_mn;             // hidden read as MN-major (N = h, K = t), box 64 x 64 (x 2)
   CUtensorMap dx_k[kDxBuffers];   // dX buffer [T, ldx], K-major, box 64 x 128
+  CUtensorMap dx_mn[kDxBuffers];  // dX buffer read as MN-major (M = v, K = t), box 64 x 64 (x 2)
   CUtensorMap dx_st[kDxBuffers];  // dX buffer written by TMA stores, box 32 x 32, no swizzle
-  CUtensorMap dxt_k[kDxBuffers];  // dXt buffer [ldx, Tp] (K = t), K-major, box 64 x 128
-  CUtensorMap dxt_st[kDxBuffers]; // dXt buffer written by TMA stores, box 32 x 32, no swizzle
 };
 
 struct BwdPlan {
@@ -82,7 +80,7 @@ struct BwdParams {
   uint32_t* err;
   float scale_log2;   // log2(e) / tau
   float inv_tau;
-  int mn3;            // w_mn is a 3-D map (one box per 128 MN columns)
+  int mn3;            // w_mn, hid_mn, dx_mn are 3-D maps (one box per 128 MN columns)
 };
 
 enum : int { kUnitR = 0, kUnitH = 1, kUnitD = 2 };

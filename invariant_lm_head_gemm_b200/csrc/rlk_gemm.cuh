@@ -193,15 +193,13 @@ struct EpiDlogits {
   }
 
   // One 128 x 256 tile, 32 columns at a time.  Each warp stages its 32 x 32
-  // bf16 block in shared memory twice, as it is and transposed (`stage`: two
-  // 2 KB buffers for each, alternating by chunk), and one lane writes them
-  // with TMA stores to dX[warp_row0 .. +32, col .. +32] and to
-  // dXt[col .. +32, warp_row0 .. +32] (rows of dX past T are not written).
-  // The caller waits for the stores (bulk_wait_all) before publishing the
-  // tile.
+  // bf16 block in shared memory (two 2 KB buffers, `stage`) and one lane
+  // writes it to dX[warp_row0 .. +32, col .. +32] with a TMA store (rows past
+  // T are not written).  The caller waits for the stores (bulk_wait_all)
+  // before publishing the tile.
   __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt,
-                              const CUtensorMap* store_map, const CUtensorMap* store_map_t,
-                              uint32_t stage, int lane, int warp_row0) {
+                              const CUtensorMap* store_map, uint32_t stage, int lane,
+                              int warp_row0) {
     const bool any_row = warp_row0 < p.T;
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
@@ -228,28 +226,19 @@ struct EpiDlogits {
       }
       if (any_row) {
         const uint32_t buf = stage + (c & 1) * 2048u;
-        const uint32_t buf_t = stage + 4096u + (c & 1) * 2048u;
-        if (lane == 0) bulk_wait_read_le1();  // the stores two chunks back have read both
+        if (lane == 0) bulk_wait_read_le1();  // the store two chunks back has read `buf`
         __syncwarp();
         const uint32_t row_addr = buf + lane * 64u;
-        uint32_t w[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) w[q] = pack_bf16x2(dx[2 * q], dx[2 * q + 1]);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          st_shared_v4(row_addr + q * 16u, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        // transposed: column j of the block becomes row j (this lane's row is
-        // column `lane` there); the same bf16 bits
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          st_shared_u16(buf_t + (2 * q) * 64u + lane * 2u, static_cast<uint16_t>(w[q] & 0xffffu));
-          st_shared_u16(buf_t + (2 * q + 1) * 64u + lane * 2u, static_cast<uint16_t>(w[q] >> 16));
-        }
+          st_shared_v4(row_addr + q * 16u, pack_bf16x2(dx[8 * q + 0], dx[8 * q + 1]),
+                       pack_bf16x2(dx[8 * q + 2], dx[8 * q + 3]),
+                       pack_bf16x2(dx[8 * q + 4], dx[8 * q + 5]),
+                       pack_bf16x2(dx[8 * q + 6], dx[8 * q + 7]));
         fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) {
           tma_store_2d(store_map, buf, loc0, warp_row0);
-          tma_store_2d(store_map_t, buf_t, warp_row0, loc0);
           bulk_commit_group();
         }
       }

@@ -32,7 +32,7 @@ namespace rlk {
 constexpr int kPStages = 6;
 constexpr uint32_t kPAStage = kBM * kBK * 2;  // this CTA's 128 rows of A: 16 KB
 constexpr uint32_t kPBStage = kBM * kBK * 2;  // this CTA's 128 rows of B: 16 KB
-constexpr uint32_t kPStaging = 4 * 8192;     // per epilogue warp: 2 x 2 KB dX + 2 x 2 KB dXt staging
+constexpr uint32_t kPStaging = 4 * 4096;     // per epilogue warp: two 2 KB store buffers
 constexpr int kRing = 4;                      // units in flight through the pair's broadcast ring
 constexpr int kPNumBars = 2 * kPStages + 5 + 2 * kRing;
 constexpr size_t kPSmemBytes =
@@ -176,12 +176,11 @@ __device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
     j.a_ext = pl.T;
     j.b_ext = pl.H;
   } else {
-    // both operands K-major (K = T): the chunk's dlogits transposed, dXt
-    // [ldx][T], and hidden transposed, hiddenT [H][T]
     j.kbs = pl.KB_D;
-    j.a_mn = j.b_mn = false;
-    j.mA = &P.maps.dxt_k[buf];
-    j.mB = &P.maps.hidt_k;
+    j.a_mn = j.b_mn = true;
+    j.mA = &P.maps.dx_mn[buf];
+    j.mB = &P.maps.hid_mn;
+    j.a3 = j.b3 = P.mn3 != 0;
     j.a_row0 = un.a * kPairM;
     j.b_col0 = un.b * kBN;
     j.a_ext = pl.ldx;
@@ -512,8 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             EpiDlogits::State st;
             EpiDlogits::begin_unit(p, st, row, 0, 0);
             EpiDlogits::tile(p, st, taddr, j.nt, &P.maps.dx_st[j.c % kDxBuffers],
-                             &P.maps.dxt_st[j.c % kDxBuffers], sStage + q * 8192u, lane,
-                             row - lane);
+                             sStage + q * 4096u, lane, row - lane);
           } else if (j.type == kUnitH) {
             EpiDh::Params p;
             p.acc = P.dh_acc;

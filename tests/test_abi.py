@@ -43,13 +43,10 @@ def test_workspace_bytes(L):
         return (x + 255) // 256 * 256
     assert fwd == 256 + 3 * a(297 * T * 4) + a(T * 4)
     # bwd: header + 3 x [T, 8192] bf16 dlogits chunk buffers + [T, H] fp32 dHidden
-    # accumulator + 3 x [8192, Tp] bf16 transposed dlogits + [H, Tp] bf16
-    # transposed hidden (Tp = T rounded up to 64) + the dependency counters
+    # accumulator + the fused backward's dependency counters
     NC, MT, NH, RT = 19, (T + 255) // 256, H // 256, 8192 // 256
-    Tp = (T + 63) // 64 * 64
     counters = NC * MT + NC * RT + NC * MT * NH + NC + 1
-    assert both == max(fwd, 256 + 3 * a(T * 8192 * 2) + a(T * H * 4) + 3 * a(8192 * Tp * 2)
-                       + a(H * Tp * 2) + a(counters * 4))
+    assert both == max(fwd, 256 + 3 * a(T * 8192 * 2) + a(T * H * 4) + a(counters * 4))
     assert binding.workspace_bytes(4, 100, 10) == 0          # H % 64 != 0
     assert binding.workspace_bytes(4, 64, 0) == 0
     assert binding.workspace_bytes(0, 64, 10) > 0
