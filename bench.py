@@ -177,6 +177,28 @@ def cpu_baseline(w, W, rows=8):
                       "forward + backward, %.1f s" % (rows, w.T, dt)}
 
 
+def cpu_oracle_sides(w, W):
+    """The oracle timed beside the other two measured paths: the forward of a
+    single row (the decode shape, T = 1) against the full head, and one
+    transition step at the report's first shape."""
+    import oracle
+    from oracle import transition as tro
+    from invariant_lm_head_gemm_b200 import workloads as wlm
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.forward(w.hidden[:1], W, w.targets[:1], w.temperature)
+    t_dec = time.perf_counter() - t0
+    B, n = wlm.TRANSITION_SHAPES[0]
+    tw = wlm.transition_case(0, B, n)
+    t0 = time.perf_counter()
+    tro.transition_sample(tw.x, tw.v, tw.eps, tw.a, tw.c, tw.s)
+    t_tr = time.perf_counter() - t0
+    return ({"us_per_call": 1e6 * t_dec, "cores": oracle.num_threads(), "kind": "oracle",
+             "sample": "fp64 C oracle forward of 1 row (H=4096, V=151936)"},
+            {"us_per_call": 1e6 * t_tr, "cores": 1, "kind": "oracle",
+             "sample": "fp64 numpy oracle, one sampling step at B3 x 257x96"})
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -489,6 +511,7 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, W_host, rows=args.cpu_rows)
+        decode["cpu_oracle"], trans["cpu_oracle"] = cpu_oracle_sides(w, W_host)
 
     if world > 1:
         dist.barrier()
