@@ -198,13 +198,13 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
   }
   auto kern = pair_kernel<Mode>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kPSmemBytes)) != cudaSuccess) {
+                           static_cast<int>(PipeCfg<Mode>::kSmemBytes)) != cudaSuccess) {
     cudaGetLastError();
     return RLK_ERR_CUDA;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kPSmemBytes;
+  cfg.dynamicSmemBytes = PipeCfg<Mode>::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;

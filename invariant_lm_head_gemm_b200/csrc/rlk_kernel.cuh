@@ -29,16 +29,24 @@
 
 namespace rlk {
 
-constexpr int kPStages = 6;
 constexpr uint32_t kPAStage = kBM * kBK * 2;  // this CTA's 128 rows of A: 16 KB
 constexpr uint32_t kPBStage = kBM * kBK * 2;  // this CTA's 128 rows of B: 16 KB
-constexpr uint32_t kPStaging = 4 * 4096;     // per epilogue warp: two 2 KB store buffers
 constexpr int kRing = 4;                      // units in flight through the pair's broadcast ring
-constexpr int kPNumBars = 2 * kPStages + 5 + 2 * kRing;
-constexpr size_t kPSmemBytes =
-    1024 + kPStages * (kPAStage + kPBStage) + kPStaging + kPNumBars * 8 + 64;
 
 enum : int { kModeFwd = 0, kModeBwd = 1, kModeGemm = 2 };
+
+// Shared memory per mode: the backward's dlogit epilogue needs 16 KB of TMA
+// store staging (two 2 KB buffers per epilogue warp) and keeps 6 operand
+// stages; the forward and the plain GEMM put that space into a 7th stage.
+template <int Mode>
+struct PipeCfg {
+  static constexpr int kStages = Mode == kModeBwd ? 6 : 7;
+  static constexpr uint32_t kStaging = Mode == kModeBwd ? 4 * 4096 : 0;
+  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kRing;
+  static constexpr size_t kSmemBytes =
+      1024 + kStages * (kPAStage + kPBStage) + kStaging + kNumBars * 8 + 64;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+};
 enum : int { kJobFwd = 3, kJobGemm = 4 };  // backward jobs use kUnitR / kUnitH / kUnitD
 
 struct FwdArgs {
@@ -223,6 +231,9 @@ __device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank
 template <int Mode>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_kernel(const __grid_constant__ typename ModeArgs<Mode>::type P) {
+  constexpr int kPStages = PipeCfg<Mode>::kStages;
+  constexpr uint32_t kPStaging = PipeCfg<Mode>::kStaging;
+  constexpr int kPNumBars = PipeCfg<Mode>::kNumBars;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
