@@ -383,10 +383,11 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
       !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM))
     return RLK_ERR_CUDA;
+  void* dx[kDxBuffers];
   for (int i = 0; i < kDxBuffers; ++i) {
-    P.dx[i] = reinterpret_cast<__nv_bfloat16*>(ws + L.dx[i]);
-    if (!map_kmajor(&P.maps.dx_k[i], P.dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !make_map(&P.maps.dx_st[i], P.dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    dx[i] = ws + L.dx[i];
+    if (!map_kmajor(&P.maps.dx_k[i], dx[i], pl.ldx, T, pl.ldx, kBM) ||
+        !make_map(&P.maps.dx_st[i], dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
       return RLK_ERR_CUDA;
   }
   // MN-major operands of the dHidden and dW units: 3-D maps (half the copies)
@@ -394,12 +395,12 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   bool mn3 = map_mnmajor3(&P.maps.w_mn, W, H, Vloc, H) &&
              map_mnmajor3(&P.maps.hid_mn, hidden, H, T, H);
   for (int i = 0; mn3 && i < kDxBuffers; ++i)
-    mn3 = map_mnmajor3(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx);
+    mn3 = map_mnmajor3(&P.maps.dx_mn[i], dx[i], pl.ldx, T, pl.ldx);
   if (!mn3) {
     if (!map_mnmajor(&P.maps.w_mn, W, H, Vloc, H) || !map_mnmajor(&P.maps.hid_mn, hidden, H, T, H))
       return RLK_ERR_CUDA;
     for (int i = 0; i < kDxBuffers; ++i)
-      if (!map_mnmajor(&P.maps.dx_mn[i], P.dx[i], pl.ldx, T, pl.ldx)) return RLK_ERR_CUDA;
+      if (!map_mnmajor(&P.maps.dx_mn[i], dx[i], pl.ldx, T, pl.ldx)) return RLK_ERR_CUDA;
   }
   P.mn3 = mn3 ? 1 : 0;
   P.targets = targets;

@@ -63,7 +63,6 @@ struct BwdParams {
   const float* entropy;
   const float* dlogp;
   const float* dentropy;
-  __nv_bfloat16* dx[kDxBuffers];
   float* dh_acc;
   __nv_bfloat16* dhidden;
   float* dh_parts;    // non-null: per-chunk dHidden products instead (EpiDh::kPart)

@@ -140,8 +140,8 @@ struct EpiFwd {
 
 // Backward recompute: the same logits tile, turned into bf16 dlogits
 //   dx = (dlogp (1[v = target] - p) - dentropy p (z - E_p z)) / tau
-// with p = 2^(y - lse log2 e), written to the chunk buffer dX[T, ldx]
-// (columns are local to the vocab chunk starting at c0).
+// with p = 2^(y - lse log2 e), written (through the store tensor map) to
+// the chunk buffer dX[T, chunk width], columns local to the chunk at c0.
 struct EpiDlogits {
   struct Params {
     const int64_t* targets;
@@ -149,12 +149,10 @@ struct EpiDlogits {
     const float* entropy;
     const float* dlogp;
     const float* dentropy;
-    __nv_bfloat16* dX;
     uint32_t* err;
     int T;
     int V;             // vocab rows of this W (a shard's own count for a shard)
-    int c0;
-    int ldx;
+    int c0;            // first W row of the chunk
     int64_t v0;        // global vocab index of this W's first row (0 unless a shard)
     int64_t Vfull;     // full vocabulary (targets are global indices)
     float scale_log2;  // log2(e) / tau

@@ -509,12 +509,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.entropy = P.entropy;
             p.dlogp = P.dlogp;
             p.dentropy = P.dentropy;
-            p.dX = P.dx[j.c % kDxBuffers];
             p.err = err;
             p.T = pl.T;
             p.V = pl.V;
             p.c0 = j.c * pl.ldx;
-            p.ldx = pl.ldx;
             p.v0 = P.v0;
             p.Vfull = P.Vfull;
             p.scale_log2 = P.scale_log2;
