@@ -113,3 +113,28 @@ def tp_linear_logp_bwd(hidden, W_shard, targets, V, temperature, lse, entropy, d
     full = torch.empty(world * R, H, dtype=torch.bfloat16, device=dev)
     dist.all_gather_into_tensor(full, mine, group=group)
     return full[:T], dW_shard
+
+
+class TPLinearLogp(torch.autograd.Function):
+    """autograd wrapper of the vocab-parallel path:
+    (logp, entropy) = TPLinearLogp.apply(hidden, W_shard, targets, V, temperature, group).
+    Every rank passes the same hidden and targets and its own shard of W
+    (rows shard_rows(V, world, rank, shard_alignment(V))); every rank gets the
+    full-vocabulary logp and entropy, the same dHidden, and the gradient of its
+    own W rows (fp32, cast to W_shard's dtype for autograd)."""
+
+    @staticmethod
+    def forward(ctx, hidden, W_shard, targets, V, temperature, group=None):
+        logp, entropy, lse = tp_linear_logp_fwd(hidden, W_shard, targets, V, temperature, group)
+        ctx.save_for_backward(hidden, W_shard, targets, lse, entropy)
+        ctx.V, ctx.temperature, ctx.group = V, temperature, group
+        return logp, entropy
+
+    @staticmethod
+    def backward(ctx, dlogp, dentropy):
+        hidden, W_shard, targets, lse, entropy = ctx.saved_tensors
+        dl = (dlogp if dlogp is not None else torch.zeros_like(lse)).float().contiguous()
+        de = (dentropy if dentropy is not None else torch.zeros_like(lse)).float().contiguous()
+        dH, dW = tp_linear_logp_bwd(hidden, W_shard, targets, ctx.V, ctx.temperature, lse,
+                                    entropy, dl, de, ctx.group)
+        return dH, dW.to(W_shard.dtype), None, None, None, None

@@ -124,3 +124,37 @@ def test_shard_grid_is_enforced():
         binding.rlk_linear_logp_bwd_shard(hid, W[512:9000].contiguous(), tg, V, 512, 1.0, lse,
                                           lse, lse, lse, dp, T)
     assert e.value.status == 2
+
+
+def test_tp_glue_on_a_one_rank_nccl_group_matches_single_gpu():
+    """The tp.py glue with its real kernels and NCCL collectives, on a group of
+    one rank (the only size one GPU can hold): logp, entropy, dHidden and dW
+    through TPLinearLogp equal LinearLogp's bit for bit."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        T, H, V, tau = 300, 256, 20000, 0.9
+        hid, W, tg, dl, de = _case(T, H, V, tau)
+        h1 = hid.clone().requires_grad_(True)
+        w1 = W.clone().requires_grad_(True)
+        lp1, en1 = tp.TPLinearLogp.apply(h1, w1, tg, V, tau)
+        (lp1 * dl + en1 * de).sum().backward()
+        h2 = hid.clone().requires_grad_(True)
+        w2 = W.clone().requires_grad_(True)
+        lp2, en2 = binding.LinearLogp.apply(h2, w2, tg, tau)
+        (lp2 * dl + en2 * de).sum().backward()
+        torch.cuda.synchronize()
+        assert torch.equal(_bits(lp1.detach()), _bits(lp2.detach()))
+        assert torch.equal(_bits(en1.detach()), _bits(en2.detach()))
+        assert torch.equal(_bits(h1.grad), _bits(h2.grad))
+        assert torch.equal(_bits(w1.grad), _bits(w2.grad))
+    finally:
+        dist.destroy_process_group()

@@ -230,3 +230,51 @@ def test_tp_backward_glue_routes_chunk_products(world, V, T):
             assert flat[g] == [1000 * src + 100 * q + 10 * k + r for r in range(R)], (q, g)
         # dHidden rows come back in rank order, the padding rows dropped
         assert dH == [float(t // R) for t in range(T)]
+
+
+def _tp_autograd_worker(rank, world, port, V, T, H, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from invariant_lm_head_gemm_b200 import tp
+    calls = []
+
+    def fake_fwd(hidden, W_shard, targets, V_, tau, group=None):
+        calls.append(("fwd", W_shard.shape[0]))
+        T_ = hidden.shape[0]
+        return (torch.full((T_,), -1.0 - rank), torch.full((T_,), 2.0), torch.full((T_,), 3.0))
+
+    def fake_bwd(hidden, W_shard, targets, V_, tau, lse, entropy, dl, de, group=None):
+        calls.append(("bwd", float(lse[0]), float(entropy[0]), float(dl[0]), float(de[0])))
+        return torch.full_like(hidden, 5.0), torch.full((W_shard.shape[0], hidden.shape[1]), 7.0)
+
+    tp.tp_linear_logp_fwd = fake_fwd
+    tp.tp_linear_logp_bwd = fake_bwd
+    h = torch.zeros(T, H, requires_grad=True)
+    w = torch.zeros(11 + rank, H, requires_grad=True)
+    logp, ent = tp.TPLinearLogp.apply(h, w, torch.zeros(T, dtype=torch.int64), V, 1.0)
+    (logp * 0.5 + ent * 0.25).sum().backward()
+    out[rank] = (calls, float(h.grad[0, 0]), list(w.grad.shape), float(w.grad[0, 0]),
+                 float(logp[0]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_tp_autograd_wrapper_plumbing():
+    world, V, T, H = 2, 20000, 3, 4
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_tp_autograd_worker, args=(world, _free_port(), V, T, H, out), nprocs=world,
+                 join=True)
+        res = dict(out)
+    for r in range(world):
+        calls, dh, wshape, dw, lp0 = res[r]
+        assert calls[0] == ("fwd", 11 + r)
+        # backward receives the saved lse / entropy and the upstream gradients
+        assert calls[1] == ("bwd", 3.0, 2.0, 0.5, 0.25)
+        assert dh == 5.0 and wshape == [11 + r, H] and dw == 7.0 and lp0 == -1.0 - r
