@@ -55,6 +55,8 @@ EDGE = [
     (3, 4096, 300, 1.0),    # long K
     (257, 192, 8193, 1.0),  # two backward chunks, the second one column wide
     (300, 256, 20000, 0.9), # three backward chunks, ragged tail
+    (33, 8192, 700, 0.25),  # long K (128 blocks) on the short-batch forward, sharp softmax
+    (300, 8192, 3000, 4.0), # long K on the pair kernels, 32 dHidden column blocks, flat softmax
 ]
 
 
