@@ -87,7 +87,11 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % index)
+        # the raw samples (the summary goes into the JSON line); directory from
+        # RLK_CLOCKS_DIR, else the system's temporary directory
+        import tempfile
+        out_dir = os.environ.get("RLK_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, "clocks_rank%d.csv" % index)
 
     def __enter__(self):
         try:
