@@ -6,9 +6,11 @@
 // 2 * 256 * H * V flops whatever T is, about as long as streaming W from
 // HBM.  Here the MMA's M side is the vocabulary (128 W rows per CTA) and its N
 // side the T rows (16, or T rounded up to 32), so the tensor work shrinks
-// with T and the kernel runs at the pace of the W stream; the shared memory
-// left over by the narrow B tiles goes to more pipeline stages, which is what
-// sets that pace (bytes of W in flight per SM).
+// with T and the kernel runs at the pace of the W stream.  That pace is set
+// by the bytes of W in flight per SM and by how long each pipeline stage is
+// held: a stage carries two K blocks, so each MMA / commit turn frees 32 KB
+// of W (one K block per stage held the stages ~20% longer for the same
+// bytes).
 //
 // Numerics are those of the pair kernel, bit for bit:
 //  * each logit is the same bf16 dot product over H in the same 64-wide K
@@ -40,7 +42,9 @@ constexpr int kDecMaxStages = 12;
 constexpr int kDecYStride = 132;    // floats per batch row of the transposed tile
 constexpr int kDecTmemCols = 256;   // two accumulators of up to 128 columns
 constexpr int kDecSplit = kDecCluster * kBM;
-constexpr uint32_t kDecABytes = kBM * kBK * 2;  // one 128 x 64 W box
+constexpr int kDecKPerStage = 2;   // K blocks per pipeline stage
+constexpr uint32_t kDecABox = kBM * kBK * 2;                    // one 128 x 64 W box
+constexpr uint32_t kDecABytes = kDecKPerStage * kDecABox;       // a stage's W boxes
 constexpr int kDecNumBars = 2 * kDecMaxStages + 9;
 
 struct DecArgs {
@@ -56,7 +60,7 @@ struct DecArgs {
 
 // Dynamic shared memory of the kernel for MMA width N and `stages` stages.
 __host__ __device__ constexpr uint32_t dec_smem_bytes(int N, int stages) {
-  return 1024u + static_cast<uint32_t>(stages) * (kDecABytes + N * kBK * 2u) +
+  return 1024u + static_cast<uint32_t>(stages) * (kDecABytes + N * kBK * 2u * kDecKPerStage) +
          static_cast<uint32_t>(N) * kDecYStride * 4u + 2u * 3u * kDecMaxRows * 4u +
          kDecNumBars * 8u + 32u;
 }
@@ -66,7 +70,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const int N = P.N, S = P.stages;
-  const uint32_t b_bytes = static_cast<uint32_t>(N) * kBK * 2u;
+  const uint32_t b_box = static_cast<uint32_t>(N) * kBK * 2u;   // one N x 64 hidden box
+  const uint32_t b_bytes = kDecKPerStage * b_box;
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + S * kDecABytes;
   float* Y = reinterpret_cast<float*>(smem + S * (kDecABytes + b_bytes));  // [N][kDecYStride]
@@ -139,16 +144,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
         if (u < 0) break;
         const int w0 = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
         const bool a_in = w0 < P.ep.V;  // a tile wholly past V is masked anyway: skip its loads
-        for (int kb = 0; kb < P.KB; ++kb) {
+        for (int kb = 0; kb < P.KB; kb += kDecKPerStage) {
+          const int nk = min(kDecKPerStage, P.KB - kb);  // K blocks in this stage
           const int s = issued % S;
           const uint32_t ph = (issued / S) & 1u;
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(s), (a_in ? kDecABytes : 0u) + b_bytes);
-          if (a_in) tma_load_2d(sA + s * kDecABytes, &P.w_k, full_bar(s), kb * kBK, w0);
-          tma_load_2d(sB + s * b_bytes, &P.hid_k, full_bar(s), kb * kBK, 0);
+          mbar_arrive_expect_tx(full_bar(s), nk * ((a_in ? kDecABox : 0u) + b_box));
+          for (int i = 0; i < nk; ++i) {
+            if (a_in)
+              tma_load_2d(sA + s * kDecABytes + i * kDecABox, &P.w_k, full_bar(s),
+                          (kb + i) * kBK, w0);
+            tma_load_2d(sB + s * b_bytes + i * b_box, &P.hid_k, full_bar(s), (kb + i) * kBK, 0);
+          }
           ++issued;
         }
       }
@@ -166,7 +176,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
         if (!mbar_wait_bounded(tempty_bar(acc), ((k >> 1) & 1u) ^ 1u, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kDecMaxRows;
-        for (int kb = 0; kb < P.KB; ++kb, ++it) {
+        for (int kb = 0; kb < P.KB; kb += kDecKPerStage, ++it) {
+          const int nk = min(kDecKPerStage, P.KB - kb);
           const int s = it % S;
           if (!mbar_wait_bounded(full_bar(s), (it / S) & 1u, abort_flag, err)) {
             ok = false;
@@ -174,11 +185,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
           }
           tc_fence_after();
           const uint32_t a_s = sA + s * kDecABytes, b_s = sB + s * b_bytes;
+          for (int i = 0; i < nk; ++i) {
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a_s + kk * 32u, 16u, 1024u);
-            const uint64_t bd = smem_desc_sw128(b_s + kk * 32u, 16u, 1024u);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(a_s + i * kDecABox + kk * 32u, 16u, 1024u);
+              const uint64_t bd = smem_desc_sw128(b_s + i * b_box + kk * 32u, 16u, 1024u);
+              umma_bf16(d_tmem, ad, bd, idesc, ((kb + i) | kk) != 0 ? 1u : 0u);
+            }
           }
           umma_commit(empty_bar(s));
         }
