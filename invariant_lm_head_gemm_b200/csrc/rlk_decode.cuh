@@ -28,7 +28,7 @@
 // Warp roles per CTA (192 threads): warp 0 producer (TMA), warp 1 MMA issuer,
 // warps 2-5 epilogue.  Two TMEM accumulators of up to 128 columns; the
 // epilogue copies an accumulator to shared memory transposed (row-major per
-// batch row) and frees it before it waits on the chain.
+// batch row), 32 rows at a time, and frees it after the last block.
 #pragma once
 
 #include "rlk_gemm.cuh"
@@ -61,7 +61,7 @@ struct DecArgs {
 // Dynamic shared memory of the kernel for MMA width N and `stages` stages.
 __host__ __device__ constexpr uint32_t dec_smem_bytes(int N, int stages) {
   return 1024u + static_cast<uint32_t>(stages) * (kDecABytes + N * kBK * 2u * kDecKPerStage) +
-         static_cast<uint32_t>(N) * kDecYStride * 4u + 2u * 3u * kDecMaxRows * 4u +
+         32u * kDecYStride * 4u + 2u * 3u * kDecMaxRows * 4u +
          kDecNumBars * 8u + 32u;
 }
 
@@ -74,14 +74,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
   const uint32_t b_bytes = kDecKPerStage * b_box;
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + S * kDecABytes;
-  float* Y = reinterpret_cast<float*>(smem + S * (kDecABytes + b_bytes));  // [N][kDecYStride]
-  float* hand = Y + N * kDecYStride;                 // [2][3][kDecMaxRows] incoming (m, s, b)
+  float* Y = reinterpret_cast<float*>(smem + S * (kDecABytes + b_bytes));  // [32][kDecYStride]
+  float* hand = Y + 32 * kDecYStride;                // [2][3][kDecMaxRows] incoming (m, s, b)
   uint64_t* bars = reinterpret_cast<uint64_t*>(hand + 2 * 3 * kDecMaxRows);
   const uint32_t bar0 = smem_u32(bars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kDecNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ok1 = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  volatile int* ok2 = reinterpret_cast<volatile int*>(tmem_slot + 3);
   volatile int* ok3 = reinterpret_cast<volatile int*>(tmem_slot + 4);
 
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -213,32 +212,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
       if (u < 0) break;
       const int acc = k & 1, h = k & 1;
       const uint32_t hph = (k >> 1) & 1u;
-      // 1. accumulator -> Y[row][W row], then free the accumulator
-      if (ep_leader) *ok1 = mbar_wait_bounded(tfull_bar(acc), hph, abort_flag, err) ? 1 : 0;
+      // 1. the accumulator, and the running triple from CTA rank-1 (or a fresh one)
+      if (ep_leader) {
+        bool ok = mbar_wait_bounded(tfull_bar(acc), hph, abort_flag, err);
+        if (ok && rank > 0) ok = mbar_wait_cluster_bounded(hfull_bar(h), hph, abort_flag, err);
+        *ok1 = ok ? 1 : 0;
+      }
       epilogue_bar();
       if (!*ok1) break;
       tc_fence_after();
-      if (N == 16) {
-        uint32_t r[16];
-        tmem_ld16(tl + acc * kDecMaxRows, r);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
-      }
-      for (int cb = 0; cb < N / 32; ++cb) {
-        uint32_t r[32];
-        tmem_ld32(tl + acc * kDecMaxRows + cb * 32, r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) Y[(cb * 32 + j) * kDecYStride + v_loc] = __uint_as_float(r[j]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
-      // 2. the running triple from CTA rank-1 (or a fresh one)
-      if (ep_leader) {
-        *ok2 = rank == 0 || mbar_wait_cluster_bounded(hfull_bar(h), hph, abort_flag, err) ? 1 : 0;
-      }
-      epilogue_bar();  // also: Y complete
-      if (!*ok2) break;
       float m = kMaskLogit, s = 0.f, b = 0.f;
       if (rank > 0) {
         mbar_try_wait_cluster(hfull_bar(h), hph);  // completed: acquire for this thread
@@ -248,23 +230,47 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
         b = in[2 * kDecMaxRows + t];
         mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
       }
-      // 3. this tile's four chunks of the split, in column order
-      if (tvalid) {
-        const int col_base = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
-        const float4* row = reinterpret_cast<const float4*>(Y + t * kDecYStride);
-#pragma unroll 1
-        for (int c = 0; c < kBM / 32; ++c) {
-          float y[32];
+      // 2. 32 batch rows at a time: their accumulator columns go to Y transposed
+      //    (all four warps, one TMEM lane quarter each), then the warp that owns
+      //    those rows folds the tile's four chunks in column order; the
+      //    accumulator is freed after its last columns are read
+      const int col_base = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
+      const int nblk = (N + 31) / 32;
+      for (int blk = 0; blk < nblk; ++blk) {
+        if (N == 16) {
+          uint32_t r[16];
+          tmem_ld16(tl + acc * kDecMaxRows, r);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 f = row[c * 8 + i];
-            y[4 * i + 0] = fwd_scale(f.x, P.ep.scale_log2);
-            y[4 * i + 1] = fwd_scale(f.y, P.ep.scale_log2);
-            y[4 * i + 2] = fwd_scale(f.z, P.ep.scale_log2);
-            y[4 * i + 3] = fwd_scale(f.w, P.ep.scale_log2);
-          }
-          fwd_chunk_update(y, col_base + c * 32, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
+          for (int j = 0; j < 16; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
+        } else {
+          uint32_t r[32];
+          tmem_ld32(tl + acc * kDecMaxRows + blk * 32, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
         }
+        if (blk == nblk - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
+        epilogue_bar();  // Y holds batch rows blk*32 .. +31
+        if (warp - 2 == blk && tvalid) {
+          const float4* row = reinterpret_cast<const float4*>(Y + lane * kDecYStride);
+#pragma unroll 1
+          for (int c = 0; c < kBM / 32; ++c) {
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 f = row[c * 8 + i];
+              y[4 * i + 0] = fwd_scale(f.x, P.ep.scale_log2);
+              y[4 * i + 1] = fwd_scale(f.y, P.ep.scale_log2);
+              y[4 * i + 2] = fwd_scale(f.z, P.ep.scale_log2);
+              y[4 * i + 3] = fwd_scale(f.w, P.ep.scale_log2);
+            }
+            fwd_chunk_update(y, col_base + c * 32, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
+          }
+        }
+        epilogue_bar();  // Y read: free for the next block
       }
       // 4. hand the triple on, or store the split's triple
       if (rank + 1 < kDecCluster) {
