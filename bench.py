@@ -330,7 +330,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         eager = 1e3 * e_a.elapsed_time(e_b) / 10
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
             call()
         for _ in range(3):
             graph.replay()
@@ -371,7 +371,7 @@ def run_ours(args):
         t_out = (torch.empty_like(tx), torch.empty_like(tx), torch.empty(Bt, device=dev))
         binding.rlk_transition_sample(tx, tv, te, ta, tc, tsd, out=t_out, workspace=t_ws)
         tg_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(tg_graph):
+        with torch.cuda.graph(tg_graph, capture_error_mode="thread_local"):
             for _ in range(20):
                 binding.rlk_transition_sample(tx, tv, te, ta, tc, tsd, out=t_out, workspace=t_ws)
         for _ in range(2):
