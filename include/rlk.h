@@ -32,8 +32,12 @@
  * (logp, entropy, lse and the dHidden row) depends only on that row's hidden
  * vector, target and gradient seeds: it is bitwise the same for any T, any
  * position of the row in the batch and any other rows in the batch, and
- * bitwise the same run to run.  dW (a sum over rows) is bitwise repeatable
- * for identical inputs: fixed summation order, no atomics.
+ * bitwise the same run to run.  (Batches of at most 128 rows run a second
+ * forward kernel, with the operands of the tensor-core product swapped; it
+ * computes every logit and every online-softmax update with the same
+ * arithmetic in the same order, and the test suite holds it to the long-batch
+ * kernel bit for bit.)  dW (a sum over rows) is bitwise repeatable for
+ * identical inputs: fixed summation order, no atomics.
  *
  * Conventions for every entry point below.
  *  - All tensor pointers are DEVICE pointers owned by the caller, row-major,
