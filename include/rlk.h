@@ -130,12 +130,17 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
  *    anything is enqueued.
  *  - The first call on a device looks up the array's device address with that
  *    device current (cudaGetSymbolAddress); make that first call before any
- *    stream capture.
+ *    stream capture.  The address is kept together with the id of the
+ *    context it belongs to: after the context is destroyed and created again
+ *    (cudaDeviceReset, or a host that releases and re-retains the primary
+ *    context) the next call looks the address up again, so that call too
+ *    belongs before any capture.  Host threads may call concurrently.
  *  - Every call shares the one array: calls whose kernels overlap on the GPU
  *    (for instance on two streams) race and corrupt each other's results.
  *    Each call clears the error word itself; an out-of-range target gives NaN
  *    logp for its row, and a timed-out internal wait turns all outputs NaN.
- *  - Calls no allocation routine of CUDA or of any other library. */
+ *  - Calls no allocation routine of CUDA or of any other library.
+ *  - Counted by rlk_call_count(0), like rlk_linear_logp_fwd. */
 rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W,
                                        const int64_t* targets, int64_t T, int64_t H, int64_t V,
                                        float temperature, float* logp, float* entropy,
@@ -296,8 +301,9 @@ rlk_status rlk_sum_ordered(const float* const* parts, int nparts, float* out, in
 /* Provenance readback, in the spirit of the pages' per-module runtime
  * readbacks (h100-cp-gradient.json, runs[].validation.runtime_readbacks:
  * backend_ids, call_count).  rlk_backend_id() names this implementation;
- * rlk_call_count(0) / (1) / (2) count successfully enqueued forward /
- * backward / self-check GEMM calls in this process. */
+ * rlk_call_count(0) / (1) / (2) count successfully enqueued forward
+ * (rlk_linear_logp_fwd and rlk_linear_logp_fwd_noalloc) / backward /
+ * self-check GEMM calls in this process. */
 const char* rlk_backend_id(void);
 uint64_t rlk_call_count(int which);
 

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -30,8 +31,11 @@ constexpr size_t kHeader = 256;  // device error word + padding
 std::atomic<uint64_t> g_calls[3];
 
 constexpr int kMaxDevices = 64;
-int g_dev_state[kMaxDevices];  // 0 unknown, 1 supported, 2 unsupported
-int g_dev_sms[kMaxDevices];
+// Per-device facts looked up on first use.  Host threads may race to fill a
+// slot (each writes the same value); the SM count is published before the
+// state that says it is valid.
+std::atomic<int> g_dev_state[kMaxDevices];  // 0 unknown, 1 supported, 2 unsupported
+std::atomic<int> g_dev_sms[kMaxDevices];
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -99,7 +103,8 @@ rlk_status check_device(int* num_sms) {
     return RLK_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return RLK_ERR_UNSUPPORTED_DEVICE;
-  if (g_dev_state[dev] == 0) {
+  int state = g_dev_state[dev].load(std::memory_order_acquire);
+  if (state == 0) {
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -107,11 +112,12 @@ rlk_status check_device(int* num_sms) {
       cudaGetLastError();
       return RLK_ERR_CUDA;
     }
-    g_dev_sms[dev] = sms;
-    g_dev_state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    state = (major == 10 && minor == 0) ? 1 : 2;
+    g_dev_sms[dev].store(sms, std::memory_order_relaxed);
+    g_dev_state[dev].store(state, std::memory_order_release);
   }
-  if (g_dev_state[dev] != 1) return RLK_ERR_UNSUPPORTED_DEVICE;
-  *num_sms = g_dev_sms[dev];
+  if (state != 1) return RLK_ERR_UNSUPPORTED_DEVICE;
+  *num_sms = g_dev_sms[dev].load(std::memory_order_relaxed);
   return RLK_OK;
 }
 
@@ -120,18 +126,20 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// A driver entry point by name, or null.
+void* driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return p;
+  cudaGetLastError();
+  return nullptr;
+}
+
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    else
-      cudaGetLastError();
-  }
+  static const EncodeTiledFn fn =
+      reinterpret_cast<EncodeTiledFn>(driver_fn("cuTensorMapEncodeTiled"));
   return fn;
 }
 
@@ -181,7 +189,7 @@ bool map_mnmajor(CUtensorMap* m, const void* base, int64_t MN, int64_t K, int64_
   return make_map(m, base, MN, K, pitch, 64, 64);
 }
 
-int g_max_clusters[3][kMaxDevices];
+std::atomic<int> g_max_clusters[3][kMaxDevices];
 
 // Launches pair_kernel<Mode> on clusters of two CTAs: at most one cluster per
 // unit and no more clusters than can be resident at once.  `cooperative`
@@ -215,7 +223,7 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int& mc = g_max_clusters[Mode][dev];
+  int mc = g_max_clusters[Mode][dev].load(std::memory_order_relaxed);
   if (mc == 0) {
     cfg.gridDim = dim3(2);
     int n = 0;
@@ -224,6 +232,7 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
       return RLK_ERR_CUDA;
     }
     mc = n;
+    g_max_clusters[Mode][dev].store(n, std::memory_order_relaxed);
   }
   cfg.numAttrs = cooperative ? 2 : 1;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<long long>(total, mc)));
@@ -240,7 +249,7 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
 // target falls in these rows, the target's scaled logit to ytgt.
 static_assert(kDecSplit == kBN * kFwdGroup, "both forward kernels must use the same splits");
 
-int g_dec_max_clusters[kDecMaxRows / 16][kMaxDevices];  // by N / 16 - 1
+std::atomic<int> g_dec_max_clusters[kDecMaxRows / 16][kMaxDevices];  // by N / 16 - 1
 
 // Forward partials for T <= kDecMaxRows (decode_fwd_kernel, rlk_decode.cuh).
 rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
@@ -291,7 +300,7 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int& mc = g_dec_max_clusters[a.N / 16 - 1][dev];
+  int mc = g_dec_max_clusters[a.N / 16 - 1][dev].load(std::memory_order_relaxed);
   if (mc == 0) {
     cfg.gridDim = dim3(kDecCluster);
     int n = 0;
@@ -300,6 +309,7 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
       return RLK_ERR_CUDA;
     }
     mc = n;
+    g_dec_max_clusters[a.N / 16 - 1][dev].store(n, std::memory_order_relaxed);
   }
   cfg.gridDim = dim3(static_cast<unsigned>(kDecCluster * std::min<int>(a.NG, mc)));
   if (cudaLaunchKernelEx(&cfg, decode_fwd_kernel, a) != cudaSuccess) {
@@ -841,9 +851,33 @@ constexpr size_t kStaticScratchBytes = size_t{32} << 20;  // 32 MiB per device
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-// Device address of g_static_scratch, looked up once per device with that
-// device current.  In host code the array's name is only a host-side stand-in.
-void* g_static_scratch_addr[kMaxDevices];
+// Device address of g_static_scratch per device, together with the id of the
+// context it was looked up in.  In host code the array's name is only a
+// host-side stand-in.  A context that is destroyed and created again (a
+// device reset) reloads this library's module, so the array may move: the
+// address is looked up again whenever the current context's id differs from
+// the one stored.  Guarded by a mutex; host threads may call concurrently.
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  void* addr;
+};
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch_slot[kMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Id of the context current on this thread; false if there is none (the
+// runtime has not bound one to this thread yet) or the driver cannot say.
+bool current_context_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_cur =
+      reinterpret_cast<CtxGetCurrentFn>(driver_fn("cuCtxGetCurrent"));
+  static const CtxGetIdFn get_id = reinterpret_cast<CtxGetIdFn>(driver_fn("cuCtxGetId"));
+  if (!get_cur || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 rlk_status static_scratch_for_current_device(void** out) {
   int dev = -1;
@@ -852,15 +886,24 @@ rlk_status static_scratch_for_current_device(void** out) {
     return RLK_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return RLK_ERR_UNSUPPORTED_DEVICE;
-  if (!g_static_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return RLK_ERR_CUDA;
-    }
-    g_static_scratch_addr[dev] = p;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchSlot& slot = g_scratch_slot[dev];
+  unsigned long long id = 0;
+  if (slot.addr && current_context_id(&id) && id == slot.ctx_id) {
+    *out = slot.addr;
+    return RLK_OK;
   }
-  *out = g_static_scratch_addr[dev];
+  // First use on this device, a new context, or no context bound to this
+  // thread yet: the lookup binds the device's primary context and returns
+  // the array's address in it.
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return RLK_ERR_CUDA;
+  }
+  slot.addr = p;
+  slot.ctx_id = current_context_id(&id) ? id : 0;
+  *out = p;
   return RLK_OK;
 }
 
@@ -913,6 +956,7 @@ rlk_status rlk_linear_logp_fwd_noalloc(const rlk_bf16* hidden, const rlk_bf16* W
   poison_on_timeout_kernel<<<std::min<int64_t>(ceil_div(T, 256), 1024), 256, 0, st>>>(
       err, logp, entropy, lse, static_cast<int>(T));
   if (cudaGetLastError() != cudaSuccess) return RLK_ERR_CUDA;
+  g_calls[0].fetch_add(1);
   return RLK_OK;
 }
 

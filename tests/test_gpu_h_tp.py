@@ -4,10 +4,18 @@ exchanged by indexing exactly as the all-gathers / all-to-all of the TP glue
 deliver them, and merged; logp, entropy, lse, dHidden and dW must equal the
 single-GPU path bit for bit for every TP degree (the pages' TP2/CP4 vs TP4/CP2
 runs agree bitwise: h100-cp-gradient.json, all_parameter_hash_comparisons,
-gradient_norm_comparisons, tokens_equal)."""
+gradient_norm_comparisons, tokens_equal), and the merged results of every
+degree must also match the fp64 oracle within the parity tolerances: logp,
+entropy and lse of every row, dHidden by relative Frobenius error, dW on
+sampled vocab rows (the pages' layouts also train correctly, not only
+identically)."""
+import functools
+
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from invariant_lm_head_gemm_b200 import binding, tp
 from tests import gpu_util as gu
 
@@ -25,6 +33,35 @@ def _case(T, H, V, tau):
     case = gu.random_case(T, H, V, tau, seed=T + V)
     return (gu.dev_bf16(case.hidden), gu.dev_bf16(case.W), gu.dev(case.targets, torch.int64),
             gu.dev(case.dlogp, torch.float32), gu.dev(case.dentropy, torch.float32))
+
+
+@functools.lru_cache(maxsize=None)
+def _oracle(T, H, V, tau):
+    """fp64 oracle results of _case(T, H, V, tau): logp, entropy, lse, dHidden,
+    and dW on sampled vocab rows (the rows' targets, both ends and a random
+    set, so that every shard of every degree holds some of them)."""
+    case = gu.random_case(T, H, V, tau, seed=T + V)
+    z = oracle.logits(case.hidden, case.W, tau)
+    lp, en, ls = oracle.softmax_stats(z, case.targets)
+    dx = oracle.dlogits(z, case.targets, tau, case.dlogp, case.dentropy)
+    dH = oracle.dhidden(dx, case.W)
+    rng = np.random.default_rng(T + H)
+    vs = np.unique(np.concatenate([case.targets, rng.choice(V, min(V, 512), replace=False),
+                                   [0, V - 1]]))
+    dW = oracle.dw(dx[:, vs], case.hidden)
+    return dict(logp=lp, entropy=en, lse=ls, dH=dH, vs=vs, dW=dW)
+
+
+def _check_fwd_against_oracle(got, ref, what):
+    for a, name in zip(got, ("logp", "entropy", "lse")):
+        gu.assert_close_vec(a.cpu().numpy(), ref[name], "%s %s" % (what, name))
+
+
+def _check_bwd_against_oracle(dH, dW, ref, what):
+    e_h = gu.rel_frob(gu.bf16_to_f64(dH), ref["dH"])
+    vs = torch.from_numpy(ref["vs"]).cuda()
+    e_w = gu.rel_frob(dW[vs].double().cpu().numpy(), ref["dW"])
+    assert e_h <= gu.FROB_TOL and e_w <= gu.FROB_TOL, (what, e_h, e_w)
 
 
 def _fwd_shards(hid, W, tg, V, tau, world, align):
@@ -47,6 +84,7 @@ def _fwd_shards(hid, W, tg, V, tau, world, align):
 def test_tp_forward_any_degree_is_single_gpu_bitwise(T, H, V):
     hid, W, tg, _, _ = _case(T, H, V, 0.9)
     ref = binding.rlk_linear_logp_fwd(hid, W, tg, 0.9)
+    oref = _oracle(T, H, V, 0.9)
     assert binding.fwd_split_width() == 512
     for world in WORLDS:
         # the forward alone needs only whole 512-row splits per shard
@@ -55,6 +93,7 @@ def test_tp_forward_any_degree_is_single_gpu_bitwise(T, H, V):
             torch.cuda.synchronize()
             for a, b, name in zip(got, ref, ("logp", "entropy", "lse")):
                 assert torch.equal(_bits(a), _bits(b)), (world, align, name)
+            _check_fwd_against_oracle(got, oref, "TP=%d align=%d" % (world, align))
 
 
 @pytest.mark.parametrize("T,H,V", SHAPES)
@@ -63,6 +102,7 @@ def test_tp_backward_any_degree_is_single_gpu_bitwise(T, H, V):
     hid, W, tg, dl, de = _case(T, H, V, tau)
     lp, en, ls = binding.rlk_linear_logp_fwd(hid, W, tg, tau)
     dH_ref, dW_ref = binding.rlk_linear_logp_bwd(hid, W, tg, tau, ls, en, dl, de)
+    oref = _oracle(T, H, V, tau)
     chunk = binding.bwd_chunk_width(V)
     assert chunk == min(8192, -(-V // 256) * 256)
     align = tp.shard_alignment(V)
@@ -88,6 +128,7 @@ def test_tp_backward_any_degree_is_single_gpu_bitwise(T, H, V):
         torch.cuda.synchronize()
         assert torch.equal(_bits(dH), _bits(dH_ref)), world
         assert torch.equal(_bits(dW), _bits(dW_ref)), world
+        _check_bwd_against_oracle(dH, dW, oref, "TP=%d" % world)
 
 
 def test_plain_part_layout_and_combine():
