@@ -84,14 +84,14 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
+    def __init__(self, index, tag=""):
         self.index = index
         self.proc = None
         # the raw samples (the summary goes into the JSON line); directory from
         # RLK_CLOCKS_DIR, else the system's temporary directory
         import tempfile
         out_dir = os.environ.get("RLK_CLOCKS_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(out_dir, "clocks_rank%d.csv" % index)
+        self.path = os.path.join(out_dir, "clocks_rank%d%s.csv" % (index, tag))
 
     def __enter__(self):
         try:
@@ -140,6 +140,27 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# Nominal dense bf16 tensor throughput per SM per clock (4096 bf16 FMAs): 148 SMs
+# at 1965 MHz give 2.38 PFLOP/s, the datasheet's 2.25 PFLOP/s at ~1.86 GHz.
+FLOPS_PER_SM_CLOCK = 8192.0
+MAX_SM_MHZ = 1965.0
+
+
+def clock_fields(ms, clk, tflops, n_sms):
+    """Clock-normalised figures of a kernel timed while `clk` sampled the SM
+    clock: its cycles per launch at the median clock, the time it would take at
+    the maximum clock, and its throughput as a fraction of the tensor peak at
+    the clock it ran at (comparable across boxes whose power-capped clocks
+    differ)."""
+    if not clk or not clk.get("sm_mhz"):
+        return {"sm_mhz": None}
+    mhz = clk["sm_mhz"]
+    return {"sm_mhz": mhz, "clock_samples": clk.get("samples"),
+            "mcycles_per_launch": ms * mhz / 1e3,
+            "ms_at_%dMHz" % MAX_SM_MHZ: ms * mhz / MAX_SM_MHZ,
+            "frac_at_clock": tflops / (n_sms * FLOPS_PER_SM_CLOCK * mhz * 1e6 / 1e12)}
 
 
 def aggregate(ms_local, tokens_local):
@@ -359,7 +380,8 @@ def run_ours(args):
     # eps; writes mean, prev_sample, logp: 20 bytes per element).  A sampler
     # loop captured whole: 20 steps in one CUDA graph, replayed 10 times.  At
     # these sizes (1.5-31 MB per step) launch gaps still set much of the time.
-    from invariant_lm_head_gemm_b200 import workloads as wlm
+    from invariant_lm_head_gemm_b200 import workloads as wl
+    wlm = wl
     trans = {"kernel": "transition_kernel (one launch per step)", "bound": "hbm",
              "unit": "GB/s", "timing": "CUDA graph of 20 steps, replayed 10 times", "shapes": [],
              "us_per_call": [], "achieved": [], "frac": []}
@@ -392,6 +414,7 @@ def run_ours(args):
         del tg_graph
 
     # ---------------------------------------------------------------- device-resident
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -412,22 +435,56 @@ def run_ours(args):
     flags = binding.rlk_read_device_error(ws)
 
     # ---------------------------------------------------------------- each pass alone
-    def per_call_ms(fn, n):
+    # Per-call CUDA events; the SM clock is sampled over each loop (at least
+    # ~0.6 s of calls, so that the 100 ms sampler sees several samples).
+    def per_call_ms(fn, n, tag):
         for _ in range(3):
             fn()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n)]
-        for a, b in ev:
-            a.record(stream)
-            fn()
-            b.record(stream)
         torch.cuda.synchronize()
-        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+        with ClockSampler(local, tag) as c:
+            for a, b in ev:
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev), c.summary()
 
-    fwd_ms = per_call_ms(lambda: binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws,
-                                                             out=(logp, ent, lse)), args.steps)
-    bwd_ms = per_call_ms(lambda: binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent, dl, de,
-                                                             ws, out=(dH, dW)), args.steps)
+    def calls_for(ms_guess, n_min):
+        return max(n_min, int(600.0 / ms_guess) + 1)
+
+    fwd_ms, fwd_clk = per_call_ms(lambda: binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws,
+                                                                      out=(logp, ent, lse)),
+                                  calls_for(5.5, args.steps), "_fwd")
+    bwd_ms, bwd_clk = per_call_ms(lambda: binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent,
+                                                                      dl, de, ws, out=(dH, dW)),
+                                  calls_for(18.0, args.steps), "_bwd")
+
+    # ---------------------------------------------------------------- the T = 4096 target point
+    # Forward + backward at T = 4096, H = 4096, V = 151936 (Qwen-shaped rows:
+    # hidden RMS-normalised, per-row dlogp ~ N(0,1), dentropy = 0.001) against
+    # the same W; and the forward alone on the same rows (the Qwen3-8B-shaped
+    # LM-head forward workload).  Device-resident inputs, W read every call.
+    tp_w = wl.target_point(2, with_weight=False)
+    T4 = tp_w.T
+    hid4 = to_dev_bf16(tp_w.hidden)
+    tg4 = torch.from_numpy(tp_w.targets).to(dev)
+    dl4 = torch.from_numpy(tp_w.dlogp).to(dev)
+    de4 = torch.from_numpy(tp_w.dentropy).to(dev)
+    outs4 = tuple(torch.empty(T4, device=dev) for _ in range(3))
+    dH4 = torch.empty(T4, H, dtype=torch.bfloat16, device=dev)
+
+    def step4():
+        binding.rlk_linear_logp_fwd(hid4, W, tg4, 1.0, ws, out=outs4)
+        binding.rlk_linear_logp_bwd(hid4, W, tg4, 1.0, outs4[2], outs4[1], dl4, de4, ws,
+                                    out=(dH4, dW))
+
+    t4_ms, t4_clk = per_call_ms(step4, calls_for(17.0, args.steps), "_t4096")
+    q_ms, q_clk = per_call_ms(lambda: binding.rlk_linear_logp_fwd(hid4, W, tg4, 1.0, ws,
+                                                                  out=outs4),
+                              calls_for(4.0, args.steps), "_qwen_fwd")
+    del hid4, dH4
 
     # ---------------------------------------------------------------- one rank of TP = 8
     # Vocab-parallel: rank 0's shard (W rows [0, 24576)) on the same batch;
@@ -444,37 +501,44 @@ def run_ours(args):
     cps = -(-(s1 - s0) // binding.bwd_chunk_width(V))
     tp_dh = torch.empty(tp_world, cps, R, H, device=dev)
     tp_dW = torch.empty(s1 - s0, H, device=dev)
-    tp_f = per_call_ms(lambda: binding.rlk_linear_logp_fwd_shard(hid, W_s, tg, V, s0, 1.0, tp_part,
-                                                                tp_yt, ws), args.steps)
-    tp_b = per_call_ms(lambda: binding.rlk_linear_logp_bwd_shard(
+    tp_f, _ = per_call_ms(lambda: binding.rlk_linear_logp_fwd_shard(hid, W_s, tg, V, s0, 1.0,
+                                                                    tp_part, tp_yt, ws),
+                          args.steps, "_tpf")
+    tp_b, _ = per_call_ms(lambda: binding.rlk_linear_logp_bwd_shard(
         hid, W_s, tg, V, s0, 1.0, lse, ent, dl, de, tp_dh, R, dW_shard=tp_dW, workspace=ws),
-        args.steps)
+        args.steps, "_tpb")
     tp_line = {"tp": tp_world, "shard_rows": s1 - s0, "fwd_shard_ms": tp_f, "bwd_shard_ms": tp_b,
                "tflops": 8.0 * T * H * (s1 - s0) / ((tp_f + tp_b) * 1e-3) / 1e12,
                "note": "rank 0's kernels on one GPU; the all-gathers / all-to-all are not "
-                       "included"}
+                       "included; with 8192-row shard alignment the largest TP = 8 shard holds "
+                       "1.29x the mean, which caps TP = 8 at 6.2x one GPU"}
     del tp_dh, tp_dW
 
     # ---------------------------------------------------------------- end to end, host buffers
     # Every step copies its inputs (hidden, targets, dlogp, dentropy) from
-    # pinned host memory and reads its result (logp, entropy) back, all inside
-    # the timed region.  The device inputs are double-buffered: step i+1's
-    # copies run on a second stream while step i computes (events keep a
-    # buffer from being overwritten before the step that reads it is done).
+    # pinned host memory and reads its results (logp, entropy and dHidden, which
+    # feeds the layer below) back to pinned host memory, all inside the timed
+    # region; dW stays on the device for the optimiser.  Inputs and results are
+    # double-buffered: the copies run on a second stream, step i+1's inputs and
+    # step i-1's results moving while step i computes (events keep a buffer set
+    # from being reused before its step and its read-back are done).
     host_in = (torch.from_numpy(w.hidden.view(np.int16)).view(torch.bfloat16).pin_memory(),
                torch.from_numpy(w.targets).pin_memory(),
                torch.from_numpy(w.dlogp).pin_memory(),
                torch.from_numpy(w.dentropy).pin_memory())
     dev_in = [(hid, tg, dl, de), tuple(torch.empty_like(t) for t in (hid, tg, dl, de))]
     res = [torch.empty(2, T, dtype=torch.float32, device=dev) for _ in range(2)]
+    dH_set = [dH, torch.empty_like(dH)]
     out_h = [torch.empty(2, T, dtype=torch.float32).pin_memory() for _ in range(2)]
+    dH_h = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     copy_stream = torch.cuda.Stream(dev)
     copied = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
     freed = [torch.cuda.Event() for _ in range(2)]
 
     def copy_in(k):
         with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(freed[k])      # the step that last read set k is done
+            copy_stream.wait_event(freed[k])      # set k's last step and read-back are done
             for d, h in zip(dev_in[k], host_in):
                 d.copy_(h, non_blocking=True)
             copied[k].record(copy_stream)
@@ -484,10 +548,14 @@ def run_ours(args):
         h_k, t_k, l_k, e_k = dev_in[k]
         binding.rlk_linear_logp_fwd(h_k, W, t_k, 1.0, ws, out=(res[k][0], res[k][1], lse))
         binding.rlk_linear_logp_bwd(h_k, W, t_k, 1.0, lse, res[k][1], l_k, e_k, ws,
-                                    out=(dH, dW))
+                                    out=(dH_set[k], dW))
         exchange()
-        out_h[k].copy_(res[k], non_blocking=True)
-        freed[k].record(stream)
+        computed[k].record(stream)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(computed[k])
+            out_h[k].copy_(res[k], non_blocking=True)
+            dH_h[k].copy_(dH_set[k], non_blocking=True)
+            freed[k].record(copy_stream)
 
     def e2e_steps(n, start_event=None):
         if start_event is not None:
@@ -497,6 +565,7 @@ def run_ours(args):
             if i + 1 < n:
                 copy_in((i + 1) % 2)
             run_set(i % 2)
+        stream.wait_event(freed[(n - 1) % 2])     # the last read-back is inside the region
 
     e2e_steps(args.warmup)
     torch.cuda.synchronize()
@@ -510,7 +579,7 @@ def run_ours(args):
     barrier()
     e2e_ms, _ = aggregate(ee0.elapsed_time(ee1) / args.steps, T)
     h2d = T * H * 2 + T * 8 + T * 4 + T * 4
-    d2h = 2 * T * 4
+    d2h = 2 * T * 4 + T * H * 2
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -529,6 +598,8 @@ def run_ours(args):
     step_tflops = flops_tok * tokens_all / world / (ms_max * 1e-3) / 1e12
     fwd_tflops = 2.0 * T * H * V / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = 6.0 * T * H * V / (bwd_ms * 1e-3) / 1e12
+    t4_tflops = flops_tok * T4 / (t4_ms * 1e-3) / 1e12
+    q_tflops = 2.0 * T4 * H * V / (q_ms * 1e-3) / 1e12
     launches_per_step = 3 + (1 if use_rs else 0)   # fwd pair kernel, combine, bwd pair
                                                     # kernel (+ the ordered sum of dW)
     value = tokens_all / (ms_max * 1e-3)
@@ -551,28 +622,50 @@ def run_ours(args):
         "pct_of_bf16_peak": {"burst": step_tflops / pk["bf16_tflops"],
                              "sustained": step_tflops / pk["bf16_tflops_sustained"],
                              "datasheet_2250": step_tflops / 2250.0, "peaks": src},
-        "roofline": {"kernel": "backward: one persistent pair-kernel launch (logits recompute + "
-                               "dlogits, dHidden and dW GEMMs), timed alone",
-                     "bound": "tensor", "achieved": bwd_tflops, "peak": pk["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": bwd_tflops / pk["bf16_tflops"],
-                     "frac_of_sustained": bwd_tflops / pk["bf16_tflops_sustained"],
-                     "traffic": bwd_traffic, "peak_source": src + " burst bf16",
-                     "flops_per_launch": 6.0 * T * H * V, "ms_per_launch": bwd_ms},
-        "fwd_roofline": {"kernel": "forward: pair-kernel GEMM + online logsumexp/entropy + "
-                                   "target gather, with its combine, timed alone",
-                         "bound": "tensor", "achieved": fwd_tflops, "peak": pk["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": fwd_tflops / pk["bf16_tflops"],
-                         "traffic": fwd_traffic, "peak_source": src + " burst bf16",
-                         "flops_per_launch": 2.0 * T * H * V, "ms_per_launch": fwd_ms},
-        "step_roofline": {"bound": "tensor", "achieved": step_tflops,
-                          "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                          "frac": step_tflops / pk["bf16_tflops_sustained"],
-                          "flops_per_token": flops_tok, "peak_source": src + " sustained bf16"},
+        "roofline": dict({"kernel": "backward: one persistent pair-kernel launch (logits "
+                                    "recompute + dlogits, dHidden and dW GEMMs), timed alone",
+                          "bound": "tensor", "achieved": bwd_tflops, "peak": pk["bf16_tflops"],
+                          "unit": "TFLOP/s", "frac": bwd_tflops / pk["bf16_tflops"],
+                          "frac_of_sustained": bwd_tflops / pk["bf16_tflops_sustained"],
+                          "traffic": bwd_traffic, "peak_source": src + " burst bf16",
+                          "flops_per_launch": 6.0 * T * H * V, "ms_per_launch": bwd_ms},
+                         **clock_fields(bwd_ms, bwd_clk, bwd_tflops, n_sms)),
+        "fwd_roofline": dict({"kernel": "forward: pair-kernel GEMM + online logsumexp/entropy + "
+                                        "target gather, with its combine, timed alone",
+                              "bound": "tensor", "achieved": fwd_tflops,
+                              "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                              "frac": fwd_tflops / pk["bf16_tflops"],
+                              "traffic": fwd_traffic, "peak_source": src + " burst bf16",
+                              "flops_per_launch": 2.0 * T * H * V, "ms_per_launch": fwd_ms},
+                             **clock_fields(fwd_ms, fwd_clk, fwd_tflops, n_sms)),
+        "step_roofline": dict({"bound": "tensor", "achieved": step_tflops,
+                               "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                               "frac": step_tflops / pk["bf16_tflops_sustained"],
+                               "flops_per_token": flops_tok,
+                               "peak_source": src + " sustained bf16", "ms_per_step": ms_max},
+                              **clock_fields(ms_max, clk.summary(), step_tflops, n_sms)),
+        "target_T4096": dict({"workload": "fwd+bwd, T=4096 Qwen-shaped rows (RMS-normalised "
+                                          "hidden, seed 2), H=4096, V=151936, tau=1",
+                              "tokens_per_s": T4 / (t4_ms * 1e-3), "ms_per_step": t4_ms,
+                              "achieved": t4_tflops, "unit": "TFLOP/s",
+                              "frac": t4_tflops / pk["bf16_tflops"],
+                              "frac_of_sustained": t4_tflops / pk["bf16_tflops_sustained"],
+                              "target_tokens_per_s": 0.6 * pk["bf16_tflops"] * 1e12 / flops_tok},
+                             **clock_fields(t4_ms, t4_clk, t4_tflops, n_sms)),
+        "qwen_fwd": dict({"workload": "Qwen3-8B-shaped LM-head forward only: T=4096 "
+                                      "(RMS-normalised hidden), H=4096, V=151936, tau=1",
+                          "tokens_per_s": T4 / (q_ms * 1e-3), "ms_per_call": q_ms,
+                          "achieved": q_tflops, "unit": "TFLOP/s",
+                          "frac": q_tflops / pk["bf16_tflops"],
+                          "target_tokens_per_s": 0.6 * pk["bf16_tflops"] * 1e12 / (2.0 * H * V)},
+                         **clock_fields(q_ms, q_clk, q_tflops, n_sms)),
         "cpu_baseline": cpu,
         "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "copies": "pinned host buffers every step; inputs double-buffered on the "
-                          "device, step i+1's copies overlap step i on a second stream"},
+                "copies": "pinned host buffers every step: hidden, targets, dlogp, dentropy in; "
+                          "logp, entropy and dHidden back; dW stays on the device for the "
+                          "optimiser; inputs and results double-buffered, copies on a second "
+                          "stream overlapping the neighbouring steps' compute"},
         "gpu_launches": launches_per_step * args.steps,
         "dw_exchange": {"included": bool(use_rs),
                         "kind": "deterministic reduce-scatter of dW: NCCL all-to-all of "
@@ -642,7 +735,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=48)
-    ap.add_argument("--ref-rows", type=int, default=2)
+    ap.add_argument("--ref-rows", type=int, default=48,
+                    help="rows of the RL step the reference arm (the fp64 oracle) runs per step")
     ap.add_argument("--no-dw-reduce", action="store_true",
                     help="N > 1: leave out the deterministic dW reduce-scatter from the step")
     ap.add_argument("--profile", choices=["fwd", "bwd", "transition"], default=None,

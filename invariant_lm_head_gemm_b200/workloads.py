@@ -150,6 +150,17 @@ def qwen_fwd(seed: int = 2, T: int = 4096, with_weight: bool = True) -> Workload
     return Workload("qwen_fwd", T, H, V, 1.0, hidden, W, targets, z, z.copy(), seed=seed)
 
 
+def target_point(seed: int = 2, T: int = 4096, with_weight: bool = True) -> Workload:
+    """Forward + backward at T=4096, H=4096, V=151936, tau = 1: the Qwen-shaped
+    rows (hidden N(0,1) then RMS-normalised, targets uniform) with per-row
+    dlogp ~ N(0,1) and dentropy = 0.001."""
+    w = qwen_fwd(seed, T, with_weight)
+    w.name = "target_point"
+    w.dlogp = _streams(seed)[_S_DLOGP].standard_normal(T).astype(np.float32)
+    w.dentropy = np.full(T, 0.001, np.float32)
+    return w
+
+
 def rl_seq_lens(seed: int, n_seq: int = 8, lo: int = 256, hi: int = 1024) -> np.ndarray:
     """8 response lengths drawn uniformly in [256, 1024] (inclusive)."""
     return _streams(seed)[_S_LENGTHS].integers(lo, hi + 1, size=n_seq, dtype=np.int64)

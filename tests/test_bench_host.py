@@ -20,3 +20,14 @@ def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
     assert bench.measured_traffic() == (None, None)
 
+
+
+def test_clock_fields_normalise_by_the_sampled_clock():
+    # 10 ms at 1500 MHz is 15 Mcycles, 7.63 ms at the 1965 MHz maximum; 1000
+    # TFLOP/s on 148 SMs at 1500 MHz is 1000 / (148 * 8192 * 1.5e9 / 1e12) of
+    # the tensor peak at that clock
+    f = bench.clock_fields(10.0, {"sm_mhz": 1500.0, "samples": 9}, 1000.0, 148)
+    assert abs(f["mcycles_per_launch"] - 15.0) < 1e-12
+    assert abs(f["ms_at_1965MHz"] - 10.0 * 1500.0 / 1965.0) < 1e-12
+    assert abs(f["frac_at_clock"] - 1000.0 / (148 * 8192 * 1.5e9 / 1e12)) < 1e-12
+    assert bench.clock_fields(10.0, None, 1000.0, 148) == {"sm_mhz": None}
