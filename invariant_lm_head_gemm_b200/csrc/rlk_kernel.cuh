@@ -6,9 +6,11 @@
 // loads rows [128 r, 128 r + 128) of the A tile and rows [128 r, 128 r + 128)
 // of the B tile (its half of N) into its own shared memory, the pair's leader
 // (rank 0) issues the MMAs, and each CTA's TMEM receives its 128 accumulator
-// rows.  Per CTA and 64-wide K block that is 16 KB of A and 16 KB of B, so a
-// six-stage TMA ring fits in shared memory and covers about 2.5k MMA cycles
-// of load latency.
+// rows.  Per CTA and 64-wide K block that is 16 KB of A and 16 KB of B.  A
+// pipeline stage holds two K blocks (64 KB per CTA, eight MMAs), and three
+// stages fit in shared memory.  The one MMA-issuing thread spends a roughly
+// fixed time per stage (its barrier wait and its commit) on top of issuing the
+// MMAs, so eight MMAs per stage keep the tensor pipe busier than four.
 //
 // Roles per CTA (192 threads): warp 0 TMA producer (both CTAs load; the
 // leader arms its "full" barrier with both CTAs' bytes and both CTAs' loads
@@ -29,18 +31,21 @@
 
 namespace rlk {
 
-constexpr uint32_t kPAStage = kBM * kBK * 2;  // this CTA's 128 rows of A: 16 KB
-constexpr uint32_t kPBStage = kBM * kBK * 2;  // this CTA's 128 rows of B: 16 KB
+constexpr uint32_t kSubA = kBM * kBK * 2;     // one K block of this CTA's 128 rows of A: 16 KB
+constexpr uint32_t kSubB = kBM * kBK * 2;     // one K block of this CTA's 128 rows of B: 16 KB
+constexpr int kSubK = 2;                      // K blocks per pipeline stage
+constexpr uint32_t kPAStage = kSubK * kSubA;  // a stage's A: 32 KB
+constexpr uint32_t kPBStage = kSubK * kSubB;  // a stage's B: 32 KB
 constexpr int kRing = 4;                      // units in flight through the pair's broadcast ring
 
 enum : int { kModeFwd = 0, kModeBwd = 1, kModeGemm = 2 };
 
-// Shared memory per mode: the backward's dlogit epilogue needs 16 KB of TMA
-// store staging (two 2 KB buffers per epilogue warp) and keeps 6 operand
-// stages; the forward and the plain GEMM put that space into a 7th stage.
+// Shared memory per mode: three operand stages (192 KB); the backward's
+// dlogit epilogue adds 16 KB of TMA store staging (two 2 KB buffers per
+// epilogue warp).
 template <int Mode>
 struct PipeCfg {
-  static constexpr int kStages = Mode == kModeBwd ? 6 : 7;
+  static constexpr int kStages = 3;
   static constexpr uint32_t kStaging = Mode == kModeBwd ? 4 * 4096 : 0;
   static constexpr int kNumBars = 2 * kStages + 5 + 2 * kRing;
   static constexpr size_t kSmemBytes =
@@ -204,12 +209,18 @@ __device__ __forceinline__ uint32_t* err_word(const FwdArgs& P) { return P.err; 
 __device__ __forceinline__ uint32_t* err_word(const GemmArgs& P) { return P.err; }
 __device__ __forceinline__ uint32_t* err_word(const BwdParams& P) { return P.err; }
 
-// Bytes CTA `rank` loads per K block of tile `t` of the job.
+// K blocks of stage `st` of a tile of `kbs` K blocks (the last stage of an odd
+// count holds one).
+__device__ __forceinline__ int stage_kblocks(int kbs, int st) {
+  return min(kSubK, kbs - st * kSubK);
+}
+
+// Bytes CTA `rank` loads per K block (not per stage) of tile `t` of the job.
 __device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank) {
   uint32_t bytes = 0;
   const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
   if (!j.a_mn) {
-    if (a0 < j.a_ext) bytes += kPAStage;
+    if (a0 < j.a_ext) bytes += kSubA;
   } else if (j.a3) {
     if (a0 < j.a_ext) bytes += 2 * kBox;  // the box counts in full, past-the-end half filled
   } else {
@@ -218,7 +229,7 @@ __device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank
   }
   const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
   if (!j.b_mn) {
-    if (b0 < j.b_ext) bytes += kPBStage;
+    if (b0 < j.b_ext) bytes += kSubB;
   } else if (j.b3) {
     if (b0 < j.b_ext) bytes += 2 * kBox;
   } else {
@@ -360,33 +371,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
           const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
           const uint32_t bytes_all = leader ? job_bytes(j, t, 0) + job_bytes(j, t, 1) : 0u;
-          for (int kb = 0; kb < j.kbs; ++kb) {
+          const int nst = (j.kbs + kSubK - 1) / kSubK;
+          for (int st = 0; st < nst; ++st) {
             const int s = issued % kPStages;
             const uint32_t ph = (issued / kPStages) & 1u;
             if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
               ok = false;
               break;
             }
+            const int nsub = stage_kblocks(j.kbs, st);
             const uint32_t fb = mapa_shared(full_bar(s), 0);
-            if (leader) mbar_arrive_expect_tx(full_bar(s), bytes_all);
-            const uint32_t dA = sA + s * kPAStage;
-            const uint32_t dB = sB + s * kPBStage;
-            const int k = kb * kBK;
-            if (!j.a_mn) {
-              if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, k, a0);
-            } else if (j.a3) {
-              if (a0 < j.a_ext) tma_load_3d_pair(dA, j.mA, fb, 0, k, a0 >> 6);
-            } else {
-              if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, a0, k);
-              if (a0 + 64 < j.a_ext) tma_load_2d_pair(dA + kBox, j.mA, fb, a0 + 64, k);
-            }
-            if (!j.b_mn) {
-              if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, k, b0);
-            } else if (j.b3) {
-              if (b0 < j.b_ext) tma_load_3d_pair(dB, j.mB, fb, 0, j.bk0 + k, b0 >> 6);
-            } else {
-              if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, b0, j.bk0 + k);
-              if (b0 + 64 < j.b_ext) tma_load_2d_pair(dB + kBox, j.mB, fb, b0 + 64, j.bk0 + k);
+            if (leader) mbar_arrive_expect_tx(full_bar(s), static_cast<uint32_t>(nsub) * bytes_all);
+            for (int sub = 0; sub < nsub; ++sub) {
+              const uint32_t dA = sA + s * kPAStage + sub * kSubA;
+              const uint32_t dB = sB + s * kPBStage + sub * kSubB;
+              const int k = (st * kSubK + sub) * kBK;
+              if (!j.a_mn) {
+                if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, k, a0);
+              } else if (j.a3) {
+                if (a0 < j.a_ext) tma_load_3d_pair(dA, j.mA, fb, 0, k, a0 >> 6);
+              } else {
+                if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, a0, k);
+                if (a0 + 64 < j.a_ext) tma_load_2d_pair(dA + kBox, j.mA, fb, a0 + 64, k);
+              }
+              if (!j.b_mn) {
+                if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, k, b0);
+              } else if (j.b3) {
+                if (b0 < j.b_ext) tma_load_3d_pair(dB, j.mB, fb, 0, j.bk0 + k, b0 >> 6);
+              } else {
+                if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, b0, j.bk0 + k);
+                if (b0 + 64 < j.b_ext) tma_load_2d_pair(dB + kBox, j.mB, fb, b0 + 64, j.bk0 + k);
+              }
             }
             ++issued;
           }
@@ -421,7 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + acc * kBN;
-          for (int kb = 0; kb < j.kbs; ++kb, ++it) {
+          const int nst = (j.kbs + kSubK - 1) / kSubK;
+          for (int st = 0; st < nst; ++st, ++it) {
             const int s = it % kPStages;
             const uint32_t ph = (it / kPStages) & 1u;
             if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
@@ -429,12 +445,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t a_s = sA + s * kPAStage, b_s = sB + s * kPBStage;
+            const int nsub = stage_kblocks(j.kbs, st);
+            for (int sub = 0; sub < nsub; ++sub) {
+              const uint32_t a_s = sA + s * kPAStage + sub * kSubA;
+              const uint32_t b_s = sB + s * kPBStage + sub * kSubB;
 #pragma unroll
-            for (int k = 0; k < kBK / 16; ++k) {
-              const uint64_t ad = smem_desc_sw128(a_s + k * a_kstep, a_lbo, 1024u);
-              const uint64_t bd = smem_desc_sw128(b_s + k * b_kstep, b_lbo, 1024u);
-              umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < kBK / 16; ++k) {
+                const uint64_t ad = smem_desc_sw128(a_s + k * a_kstep, a_lbo, 1024u);
+                const uint64_t bd = smem_desc_sw128(b_s + k * b_kstep, b_lbo, 1024u);
+                umma_bf16_pair(d_tmem, ad, bd, idesc, (st | sub | k) != 0 ? 1u : 0u);
+              }
             }
             umma_commit_pair_both(empty_bar(s));
           }
