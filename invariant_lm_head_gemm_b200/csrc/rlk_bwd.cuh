@@ -94,16 +94,14 @@ __host__ __device__ inline int bwd_chunk_valid(const BwdPlan& P, int c) {
 __host__ __device__ inline int bwd_rt(const BwdPlan& P, int c) {
   return c == P.NC - 1 ? P.RT_last : P.RT_full;
 }
-__host__ __device__ inline long long bwd_nR(const BwdPlan& P, int c) {
-  return static_cast<long long>(P.MT) * bwd_rt(P, c);
+// Unit counts and unit decoding use 32-bit arithmetic: the host rejects any
+// plan with 2^31 units or more (bwd_total_units counts in 64 bits).
+__host__ __device__ inline int bwd_nR(const BwdPlan& P, int c) { return P.MT * bwd_rt(P, c); }
+__host__ __device__ inline int bwd_nH(const BwdPlan& P) { return P.MT * P.NH; }
+__host__ __device__ inline int bwd_nD(const BwdPlan& P, int c) {
+  return P.NH * (c == P.NC - 1 ? P.VT_last : P.VT_full);
 }
-__host__ __device__ inline long long bwd_nH(const BwdPlan& P) {
-  return static_cast<long long>(P.MT) * P.NH;
-}
-__host__ __device__ inline long long bwd_nD(const BwdPlan& P, int c) {
-  return static_cast<long long>(P.NH) * (c == P.NC - 1 ? P.VT_last : P.VT_full);
-}
-__host__ __device__ inline long long bwd_group_size(const BwdPlan& P, int g) {
+__host__ __device__ inline int bwd_group_size(const BwdPlan& P, int g) {
   return bwd_nH(P) + bwd_nD(P, g) + (g + 2 < P.NC ? bwd_nR(P, g + 2) : 0);
 }
 
@@ -132,14 +130,19 @@ __host__ inline BwdPlan make_bwd_plan(int64_t T, int64_t H, int64_t V, int64_t l
 }
 
 __host__ inline long long bwd_total_units(const BwdPlan& P) {
+  // every chunk contributes its R, H and D units once
   long long t = 0;
-  for (int c = 0; c < 2 && c < P.NC; ++c) t += bwd_nR(P, c);
-  for (int g = 0; g < P.NC; ++g) t += bwd_group_size(P, g);
+  for (int c = 0; c < P.NC; ++c) {
+    const long long rt = c == P.NC - 1 ? P.RT_last : P.RT_full;
+    const long long vt = c == P.NC - 1 ? P.VT_last : P.VT_full;
+    t += static_cast<long long>(P.MT) * rt + static_cast<long long>(P.MT) * P.NH +
+         static_cast<long long>(P.NH) * vt;
+  }
   return t;
 }
 
-__host__ __device__ inline BwdUnit bwd_seg_R(const BwdPlan& P, int c, long long i) {
-  return BwdUnit{kUnitR, c, static_cast<int>(i % P.MT), static_cast<int>(i / P.MT)};
+__host__ __device__ inline BwdUnit bwd_seg_R(const BwdPlan& P, int c, int i) {
+  return BwdUnit{kUnitR, c, i % P.MT, i / P.MT};
 }
 // dHidden units of one chunk in groups of kHGroup row blocks: inside a group
 // the row block varies fastest, then the column block.  The units in flight
@@ -147,53 +150,52 @@ __host__ __device__ inline BwdUnit bwd_seg_R(const BwdPlan& P, int c, long long 
 // chunk's W columns nor its dX rows have to stream from DRAM many times.
 constexpr int kHGroup = 8;
 
-__host__ __device__ inline BwdUnit bwd_seg_H(const BwdPlan& P, int c, long long i) {
-  const long long full = P.MT / kHGroup;
-  const long long per_group = static_cast<long long>(kHGroup) * P.NH;
+__host__ __device__ inline BwdUnit bwd_seg_H(const BwdPlan& P, int c, int i) {
+  const int full = P.MT / kHGroup;
+  const int per_group = kHGroup * P.NH;
   int m, n;
   if (i < full * per_group) {
-    const long long g = i / per_group, r = i % per_group;
-    n = static_cast<int>(r / kHGroup);
-    m = static_cast<int>(g * kHGroup + r % kHGroup);
+    const int g = i / per_group, r = i % per_group;
+    n = r / kHGroup;
+    m = g * kHGroup + r % kHGroup;
   } else {
     const int rem = P.MT % kHGroup;
-    const long long r = i - full * per_group;
-    n = static_cast<int>(r / rem);
-    m = static_cast<int>(full * kHGroup + r % rem);
+    const int r = i - full * per_group;
+    n = r / rem;
+    m = full * kHGroup + r % rem;
   }
   return BwdUnit{kUnitH, c, m, n};
 }
-__host__ __device__ inline BwdUnit bwd_seg_D(const BwdPlan& P, int c, long long i) {
-  return BwdUnit{kUnitD, c, static_cast<int>(i / P.NH), static_cast<int>(i % P.NH)};
+__host__ __device__ inline BwdUnit bwd_seg_D(const BwdPlan& P, int c, int i) {
+  return BwdUnit{kUnitD, c, i / P.NH, i % P.NH};
 }
 
 // Unit r of group g: H(g), then D(g), then R(g + 2).
-__host__ __device__ inline BwdUnit bwd_group_unit(const BwdPlan& P, int g, long long r) {
-  const long long h = bwd_nH(P);
+__host__ __device__ inline BwdUnit bwd_group_unit(const BwdPlan& P, int g, int r) {
+  const int h = bwd_nH(P);
   if (r < h) return bwd_seg_H(P, g, r);
   r -= h;
-  const long long d = bwd_nD(P, g);
+  const int d = bwd_nD(P, g);
   if (r < d) return bwd_seg_D(P, g, r);
   return bwd_seg_R(P, g + 2, r - d);
 }
 
-__host__ __device__ inline BwdUnit bwd_decode(const BwdPlan& P, long long u) {
+__host__ __device__ inline BwdUnit bwd_decode(const BwdPlan& P, int u) {
   for (int c = 0; c < 2 && c < P.NC; ++c) {
-    const long long n = bwd_nR(P, c);
+    const int n = bwd_nR(P, c);
     if (u < n) return bwd_seg_R(P, c, u);
     u -= n;
   }
   // groups 0 .. NC-4 involve full chunks only and all have the same size
   const int nreg = P.NC > 3 ? P.NC - 3 : 0;
-  const long long gs = bwd_nH(P) + static_cast<long long>(P.NH) * P.VT_full +
-                       static_cast<long long>(P.MT) * P.RT_full;
+  const int gs = bwd_nH(P) + P.NH * P.VT_full + P.MT * P.RT_full;
   if (u < nreg * gs) {
-    const int g = static_cast<int>(u / gs);
+    const int g = u / gs;
     return bwd_group_unit(P, g, u - g * gs);
   }
   u -= nreg * gs;
   for (int g = nreg; g < P.NC; ++g) {
-    const long long n = bwd_group_size(P, g);
+    const int n = bwd_group_size(P, g);
     if (u < n) return bwd_group_unit(P, g, u);
     u -= n;
   }

@@ -157,7 +157,7 @@ __device__ __forceinline__ Job make_job(const GemmArgs& P, long long u) {
 
 __device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
   const BwdPlan& pl = P.plan;
-  const BwdUnit un = bwd_decode(pl, u);
+  const BwdUnit un = bwd_decode(pl, static_cast<int>(u));
   Job j;
   j.type = un.type;
   j.c = un.c;
@@ -322,11 +322,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive_cluster(mapa_shared(sempty_bar(slot), 0));
     return v;
   };
-  auto claim_unit = [&](uint32_t k) -> long long {
+  // The leader's producer claims each unit one unit ahead of publishing it
+  // (the claim's atomic then runs while the current unit's copies are issued),
+  // and publishes unit k in ring slot k % kRing.  Claiming ahead keeps the
+  // order ascending, and a claimed unit is always processed by a running pair.
+  auto publish_unit = [&](uint32_t k, long long u) -> long long {
     const int slot = k % kRing;
     if (!mbar_wait_bounded(sempty_bar(slot), ((k / kRing) & 1u) ^ 1u, abort_flag, err)) return -1;
-    long long u = -1;
-    if constexpr (kDynamic) u = atomicAdd(P.next_unit, 1u);
     if (u >= total) u = -1;
     st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 0), static_cast<uint32_t>(u));
     st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 1), static_cast<uint32_t>(u));
@@ -340,10 +342,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
+      uint32_t claimed = 0;
+      if constexpr (kDynamic) {
+        if (leader) claimed = atomicAdd(P.next_unit, 1u);
+      }
       for (uint32_t k = 0; ok; ++k) {
         long long u;
         if constexpr (kDynamic) {
-          u = leader ? claim_unit(k) : fetch_unit(k);
+          if (leader) {
+            u = publish_unit(k, claimed);
+            if (u >= 0) claimed = atomicAdd(P.next_unit, 1u);
+          } else {
+            u = fetch_unit(k);
+          }
         } else {
           u = static_unit(k);
         }
