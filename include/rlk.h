@@ -311,6 +311,29 @@ uint64_t rlk_call_count(int which);
  * then clears it.  Synchronises `stream`. */
 rlk_status rlk_read_device_error(void* workspace, uint32_t* flags, void* stream);
 
+/* Test hook for the fail-closed path; not for production use.  The pages' runs
+ * require an error status rather than a hang when the operator cannot finish
+ * (VIME Qwen3-8B TP4/CP2 page, "Required gates"; h3-runtime-integration-b200
+ * report, runtime mode fail_on_fallback).  Every wait inside the kernels is
+ * bounded; when one gives up, the kernel sets RLK_DEVERR_TIMEOUT in the
+ * workspace's error word, lets its in-flight copies and MMAs finish, frees its
+ * tensor memory and returns, and the outputs are not to be used.
+ * rlk_test_linear_logp_bwd_stall is rlk_linear_logp_bwd (same arguments,
+ * layouts and ownership) with two more: wait_limit_ns bounds every wait of the
+ * launch (1 ms .. 2 s; the production entry points use 2 s), and stall != 0
+ * makes the first dHidden unit wait for one more recompute tile than exists,
+ * a dependency nothing ever meets.  With stall set the call still returns
+ * RLK_OK (the launch is enqueued); rlk_read_device_error then reports
+ * RLK_DEVERR_TIMEOUT, and later calls on the same workspace and stream behave
+ * as on a fresh one.  T = 0 or a limit outside the range: RLK_ERR_INVALID_ARG. */
+rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16* W,
+                                          const int64_t* targets, int64_t T, int64_t H,
+                                          int64_t V, float temperature, const float* lse,
+                                          const float* entropy, const float* dlogp,
+                                          const float* dentropy, rlk_bf16* dHidden, float* dW,
+                                          void* workspace, size_t workspace_bytes,
+                                          uint64_t wait_limit_ns, int stall, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* rlk_status_string(rlk_status status);
 

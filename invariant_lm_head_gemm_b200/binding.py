@@ -159,6 +159,33 @@ def rlk_linear_logp_bwd(hidden, W, targets, temperature, lse, entropy, dlogp, de
     return dHidden, dW
 
 
+_stall_fn = None
+
+
+def rlk_test_linear_logp_bwd_stall(hidden, W, targets, temperature, lse, entropy, dlogp,
+                                   dentropy, workspace, out, wait_limit_ns, stall,
+                                   stream=None):
+    """Test hook of the fail-closed path: the backward with every wait bounded
+    by wait_limit_ns and, when stall is set, one dependency that is never met
+    (the device error word then reports RLK_DEVERR_TIMEOUT)."""
+    global _stall_fn
+    if _stall_fn is None:
+        f = lib().rlk_test_linear_logp_bwd_stall
+        f.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, _P, _P,
+                      ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, _P]
+        f.restype = ctypes.c_int
+        _stall_fn = f
+    T, H = hidden.shape
+    V = W.shape[0]
+    dHidden, dW = out
+    _check(_stall_fn(_ptr(hidden), _ptr(W), _ptr(targets), T, H, V, float(temperature), _ptr(lse),
+                     _ptr(entropy), _ptr(dlogp), _ptr(dentropy), _ptr(dHidden), _ptr(dW),
+                     _ptr(workspace), workspace.numel(), int(wait_limit_ns), int(stall),
+                     _stream(stream)),
+           "rlk_test_linear_logp_bwd_stall")
+    return dHidden, dW
+
+
 def rlk_gemm_bf16_f32(A, B, a_mn_major=False, b_mn_major=False, stream=None):
     """C = A' . B'^T through the tensor-core mainloop (self-check entry).
     A' is A ([M,K]) or A^T (A stored [K,M] when a_mn_major); B' likewise."""

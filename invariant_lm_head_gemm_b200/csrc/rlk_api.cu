@@ -386,7 +386,8 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
                        float temperature, const float* lse, const float* entropy,
                        const float* dlogp, const float* dentropy, rlk_bf16* dHidden,
                        float* dh_parts, int64_t part_rows, int64_t part_chunks, float* dW,
-                       uint8_t* ws, const Layout& L, cudaStream_t st) {
+                       uint8_t* ws, const Layout& L, cudaStream_t st,
+                       uint64_t wait_limit_ns = kWaitLimitNs, int stall_first_h = 0) {
   BwdParams P;
   P.plan = make_bwd_plan(T, H, Vloc, vchunk(Vfull));
   const BwdPlan& pl = P.plan;
@@ -436,6 +437,8 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   P.err = reinterpret_cast<uint32_t*>(ws);
   P.scale_log2 = kLog2e / temperature;
   P.inv_tau = 1.0f / temperature;
+  P.wait_limit_ns = wait_limit_ns;
+  P.stall_first_h = stall_first_h;
 
   if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
   // Units wait on units claimed earlier, and only running CTA pairs claim
@@ -520,6 +523,35 @@ rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
     return s;
   g_calls[1].fetch_add(1);
   return RLK_OK;
+}
+
+// Test hook (declared in rlk.h): the backward with a chosen bound on every
+// wait and, optionally, one dependency that is never met.
+rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16* W,
+                                          const int64_t* targets, int64_t T, int64_t H,
+                                          int64_t V, float temperature, const float* lse,
+                                          const float* entropy, const float* dlogp,
+                                          const float* dentropy, rlk_bf16* dHidden, float* dW,
+                                          void* workspace, size_t workspace_bytes,
+                                          uint64_t wait_limit_ns, int stall, void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (T == 0 || wait_limit_ns < 1000000ull || wait_limit_ns > kWaitLimitNs)
+    return RLK_ERR_INVALID_ARG;  // 1 ms .. 2 s
+  if (!hidden || !W || !targets || !lse || !entropy || !dlogp || !dentropy || !dHidden || !dW ||
+      !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(dHidden, 16) || !aligned(dW, 16) ||
+      !aligned(workspace, 256) || !aligned(targets, 8) || !aligned(lse, 4) ||
+      !aligned(entropy, 4) || !aligned(dlogp, 4) || !aligned(dentropy, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);
+  if (workspace_bytes < L.bwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  return enqueue_bwd(hidden, W, targets, T, H, V, 0, V, temperature, lse, entropy, dlogp,
+                     dentropy, dHidden, nullptr, 0, 0, dW, static_cast<uint8_t*>(workspace), L,
+                     static_cast<cudaStream_t>(stream), wait_limit_ns, stall != 0 ? 1 : 0);
 }
 
 size_t rlk_gemm_workspace_bytes(void) { return kHeader; }

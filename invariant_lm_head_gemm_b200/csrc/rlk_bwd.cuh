@@ -80,6 +80,8 @@ struct BwdParams {
   float scale_log2;   // log2(e) / tau
   float inv_tau;
   int mn3;            // w_mn, hid_mn, dx_mn are 3-D maps (one box per 128 MN columns)
+  uint64_t wait_limit_ns;  // bound of every wait (kWaitLimitNs outside the test hook)
+  int stall_first_h;  // test hook: the first dHidden unit waits for one R unit too many
 };
 
 enum : int { kUnitR = 0, kUnitH = 1, kUnitD = 2 };

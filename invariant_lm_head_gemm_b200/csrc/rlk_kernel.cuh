@@ -208,6 +208,9 @@ __device__ __forceinline__ long long total_units(const BwdParams& P) { return P.
 __device__ __forceinline__ uint32_t* err_word(const FwdArgs& P) { return P.err; }
 __device__ __forceinline__ uint32_t* err_word(const GemmArgs& P) { return P.err; }
 __device__ __forceinline__ uint32_t* err_word(const BwdParams& P) { return P.err; }
+__device__ __forceinline__ uint64_t wait_limit(const FwdArgs&) { return kWaitLimitNs; }
+__device__ __forceinline__ uint64_t wait_limit(const GemmArgs&) { return kWaitLimitNs; }
+__device__ __forceinline__ uint64_t wait_limit(const BwdParams& P) { return P.wait_limit_ns; }
 
 // K blocks of stage `st` of a tile of `kbs` K blocks (the last stage of an odd
 // count holds one).
@@ -274,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long npairs = gridDim.x >> 1;
   const long long total = total_units(P);
   uint32_t* err = err_word(P);
+  const uint64_t lim = wait_limit(P);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto fetch_unit = [&](uint32_t k) -> long long {
     const int slot = k % kRing;
-    if (!mbar_wait_cluster_bounded(sfull_bar(slot), (k / kRing) & 1u, abort_flag, err)) return -1;
+    if (!mbar_wait_cluster_bounded(sfull_bar(slot), (k / kRing) & 1u, abort_flag, err, lim)) return -1;
     const int v = static_cast<int>(ld_shared_u32(ring_addr + 4u * slot));
     mbar_arrive_cluster(mapa_shared(sempty_bar(slot), 0));
     return v;
@@ -328,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // order ascending, and a claimed unit is always processed by a running pair.
   auto publish_unit = [&](uint32_t k, long long u) -> long long {
     const int slot = k % kRing;
-    if (!mbar_wait_bounded(sempty_bar(slot), ((k / kRing) & 1u) ^ 1u, abort_flag, err)) return -1;
+    if (!mbar_wait_bounded(sempty_bar(slot), ((k / kRing) & 1u) ^ 1u, abort_flag, err, lim)) return -1;
     if (u >= total) u = -1;
     st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 0), static_cast<uint32_t>(u));
     st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 1), static_cast<uint32_t>(u));
@@ -364,12 +368,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (Mode == kModeBwd) {
           const BwdPlan& pl = P.plan;
           if (j.type == kUnitH) {
+            // the test hook asks one unit too many of the first dHidden unit
+            const uint32_t extra =
+                P.stall_first_h != 0 && j.c == 0 && j.mt == 0 && j.nt == 0 ? 1u : 0u;
             ok = wait_counter_bounded(P.rdone_m + static_cast<size_t>(j.c) * pl.MT + j.mt,
-                                      2u * static_cast<uint32_t>(bwd_rt(pl, j.c)), abort_flag,
-                                      err);
+                                      2u * static_cast<uint32_t>(bwd_rt(pl, j.c)) + extra,
+                                      abort_flag, err, lim);
           } else if (j.type == kUnitD) {
             ok = wait_counter_bounded(P.rdone_j + static_cast<size_t>(j.c) * pl.RT_full + j.mt,
-                                      2u * static_cast<uint32_t>(pl.MT), abort_flag, err);
+                                      2u * static_cast<uint32_t>(pl.MT), abort_flag, err, lim);
           }
           if (!ok) break;
           if (j.type != kUnitR) fence_proxy_async_global();
@@ -386,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int st = 0; st < nst; ++st) {
             const int s = issued % kPStages;
             const uint32_t ph = (issued / kPStages) & 1u;
-            if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
+            if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err, lim)) {
               ok = false;
               break;
             }
@@ -441,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; ok && t < j.ntiles; ++t, ++tc) {
           const int acc = tc & 1;
           const uint32_t use = tc >> 1;
-          if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, err)) {
+          if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, err, lim)) {
             ok = false;
             break;
           }
@@ -451,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int st = 0; st < nst; ++st, ++it) {
             const int s = it % kPStages;
             const uint32_t ph = (it / kPStages) & 1u;
-            if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
+            if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err, lim)) {
               ok = false;
               break;
             }
@@ -500,19 +507,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int acc = tc & 1;
         const uint32_t use = tc >> 1;
         if (ep_leader) {
-          bool ok = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, err);
+          bool ok = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, err, lim);
           if constexpr (Mode == kModeBwd) {
             const BwdPlan& pl = P.plan;
             if (ok && j.type == kUnitR && j.c >= kDxBuffers) {
               const int c3 = j.c - kDxBuffers;
               ok = wait_counter_bounded(P.bufdone + c3,
                                         2u * static_cast<uint32_t>(bwd_nH(pl) + bwd_nD(pl, c3)),
-                                        abort_flag, err);
+                                        abort_flag, err, lim);
             }
             if (ok && j.type == kUnitH && j.c >= 1) {
               ok = wait_counter_bounded(
                   P.hdone + (static_cast<size_t>(j.c - 1) * pl.MT + j.mt) * pl.NH + j.nt, 2u,
-                  abort_flag, err);
+                  abort_flag, err, lim);
             }
           }
           *ep_ok = ok ? 1 : 0;

@@ -61,17 +61,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits until the phase with the given parity of `bar` has completed.
 // Returns false (and raises the CTA's abort flag and the device error word)
-// when the wait exceeds kWaitLimitNs, or false at once when another role of
-// the CTA has already aborted.
+// when the wait exceeds `limit_ns` (kWaitLimitNs unless a caller passes a
+// shorter limit), or false at once when another role of the CTA has already
+// aborted.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint32_t* err) {
+                                                  volatile int* abort_flag, uint32_t* err,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(err, kDevErrTimeout);
         return false;
@@ -234,7 +236,8 @@ __device__ __forceinline__ void epilogue_bar() {
 
 // Waits until *p >= target (acquire).  Bounded like mbar_wait_bounded.
 __device__ __forceinline__ bool wait_counter_bounded(const uint32_t* p, uint32_t target,
-                                                     volatile int* abort_flag, uint32_t* err) {
+                                                     volatile int* abort_flag, uint32_t* err,
+                                                     uint64_t limit_ns = kWaitLimitNs) {
   if (ld_acquire_gpu(p) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -242,7 +245,7 @@ __device__ __forceinline__ bool wait_counter_bounded(const uint32_t* p, uint32_t
     if (ld_acquire_gpu(p) >= target) return true;
     if ((i & 15u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(err, kDevErrTimeout);
         return false;
@@ -404,14 +407,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // mbar_wait_bounded with cluster-scope acquire (the phase may have been
 // completed by the other CTA of the pair).
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity,
-                                                          volatile int* abort_flag, uint32_t* err) {
+                                                          volatile int* abort_flag, uint32_t* err,
+                                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(err, kDevErrTimeout);
         return false;

@@ -227,3 +227,18 @@ def test_transition_argument_errors(L):
     lg = L.rlk_transition_logp
     assert lg(A16, A16, None, A16, A16, A16, 3, 24672, None, A16, A256, need, None) == INVALID
     assert lg(A16, A16, A16, A16, A16, A16, 3, 10, None, A16, A256, need, None) == SHAPE
+
+
+def test_stall_hook_rejects_limits_outside_its_range(L):
+    """The fail-closed test hook checks its wait bound (1 ms .. 2 s) before
+    anything touches the device: these pointers are never dereferenced."""
+    f = L.rlk_test_linear_logp_bwd_stall
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_float] + \
+        [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    p = 0x10000
+    args = [p, p, p, 4, 64, 100, 1.0, p, p, p, p, p, p, p, 1 << 20]
+    assert f(*args, 10, 1, None) == INVALID               # below 1 ms
+    assert f(*args, 3_000_000_000, 1, None) == INVALID    # above 2 s
+    assert f(p, p, p, 0, 64, 100, 1.0, p, p, p, p, p, p, p, 1 << 20, 100_000_000, 1,
+             None) == INVALID                              # T = 0
