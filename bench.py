@@ -691,6 +691,23 @@ def run_profile(args):
     from invariant_lm_head_gemm_b200 import binding
     from invariant_lm_head_gemm_b200 import workloads as wl
 
+    if args.profile == "cublas":
+        # The library GEMM beside the pair kernel for a like-for-like capture:
+        # torch.matmul (cuBLAS) bf16 at the forward's shape, hidden . W^T
+        # (T x V x H), and at 8192^3.  Nothing of the operator runs here.
+        dev = torch.device("cuda", 0)
+        T, H, V = args.T, 4096, args.V
+        g = torch.Generator(device="cpu").manual_seed(5)
+        hid = torch.randn(T, H, generator=g).to(torch.bfloat16).to(dev)
+        W = (0.02 * torch.randn(V, H, generator=g)).to(torch.bfloat16).to(dev)
+        a = torch.randn(8192, 8192, generator=g).to(torch.bfloat16).to(dev)
+        for _ in range(args.iters):
+            hid @ W.t()
+            a @ a
+        torch.cuda.synchronize()
+        print("profile case done: cublas T=%d H=%d V=%d and 8192^3, iters=%d" % (
+            T, H, V, args.iters))
+        return 0
     if args.profile == "transition":
         B, n = wl.TRANSITION_SHAPES[1]
         tw = wl.transition_case(1, B, n)
@@ -739,7 +756,7 @@ def main():
                     help="rows of the RL step the reference arm (the fp64 oracle) runs per step")
     ap.add_argument("--no-dw-reduce", action="store_true",
                     help="N > 1: leave out the deterministic dW reduce-scatter from the step")
-    ap.add_argument("--profile", choices=["fwd", "bwd", "transition"], default=None,
+    ap.add_argument("--profile", choices=["fwd", "bwd", "transition", "cublas"], default=None,
                     help="run a small case for an ncu capture instead of the benchmark")
     ap.add_argument("--T", type=int, default=2048, help="rows of the --profile case")
     ap.add_argument("--V", type=int, default=32768, help="vocab of the --profile case")
