@@ -304,22 +304,49 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     # N > 1: the data-parallel exchange of dW (deterministic reduce-scatter:
-    # one NCCL all-to-all of vocab slices, then the rank-ordered sum)
+    # NCCL all-to-all of vocab slices, then the rank-ordered sum).  Overlapped
+    # (default): the backward publishes each vocab chunk's completion and the
+    # exchange runs a group of chunks at a time on a second stream, each group
+    # waiting on the device for its chunks; "after": one exchange once the
+    # backward is done.
     use_rs = world > 1 and not args.no_dw_reduce
+    overlap = use_rs and args.dw_exchange == "overlap"
+    chunk = binding.bwd_chunk_width(V)
+    groups = -(-(-(-V // chunk)) // args.dw_group_chunks)
     if use_rs:
         from invariant_lm_head_gemm_b200 import dp
         per = -(-V // world)
         rs_recv = torch.empty(world, per, H, dtype=torch.float32, device=dev)
-        rs_out = torch.empty(per, H, dtype=torch.float32, device=dev)
+        # a rank's rows of the group-wise exchange exceed V / world by at most
+        # one per group
+        rs_out = torch.empty(per + groups, H, dtype=torch.float32, device=dev)
+        comm = torch.cuda.Stream(dev)
+        words = torch.zeros(-(-V // chunk), dtype=torch.int32, device=dev)
+        seq = [0]
 
-    def exchange():
-        if use_rs:
-            dp.reduce_scatter_dw(dW, rs_recv, rs_out)
+    def backward(h, t, l_, e_, dlp, den, out):
+        """The backward and, for N > 1, the dW exchange it feeds."""
+        if not use_rs:
+            binding.rlk_linear_logp_bwd(h, W, t, 1.0, l_, e_, dlp, den, ws, out=out)
+        elif overlap:
+            stream.wait_stream(comm)       # the last exchange has read dW
+            seq[0] += 1
+            binding.rlk_linear_logp_bwd_signal(h, W, t, 1.0, l_, e_, dlp, den, ws, out, words,
+                                               seq[0])
+            dp.reduce_scatter_dw_overlapped(out[1], chunk, chunk_done=words, seq=seq[0],
+                                            group_chunks=args.dw_group_chunks, stream=comm,
+                                            recv=rs_recv.view(-1), out=rs_out)
+        else:
+            binding.rlk_linear_logp_bwd(h, W, t, 1.0, l_, e_, dlp, den, ws, out=out)
+            dp.reduce_scatter_dw(out[1], rs_recv, rs_out)
+
+    def join_exchange():
+        if overlap:
+            stream.wait_stream(comm)
 
     def step():
         binding.rlk_linear_logp_fwd(hid, W, tg, 1.0, ws, out=(logp, ent, lse))
-        binding.rlk_linear_logp_bwd(hid, W, tg, 1.0, lse, ent, dl, de, ws, out=(dH, dW))
-        exchange()
+        backward(hid, tg, lse, ent, dl, de, (dH, dW))
 
     def barrier():
         if world > 1:
@@ -426,6 +453,7 @@ def run_ours(args):
         e0.record(stream)
         for _ in range(args.steps):
             step()
+        join_exchange()
         e1.record(stream)
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_pop()
@@ -547,9 +575,7 @@ def run_ours(args):
         stream.wait_event(copied[k])
         h_k, t_k, l_k, e_k = dev_in[k]
         binding.rlk_linear_logp_fwd(h_k, W, t_k, 1.0, ws, out=(res[k][0], res[k][1], lse))
-        binding.rlk_linear_logp_bwd(h_k, W, t_k, 1.0, lse, res[k][1], l_k, e_k, ws,
-                                    out=(dH_set[k], dW))
-        exchange()
+        backward(h_k, t_k, lse, res[k][1], l_k, e_k, (dH_set[k], dW))
         computed[k].record(stream)
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(computed[k])
@@ -565,6 +591,7 @@ def run_ours(args):
             if i + 1 < n:
                 copy_in((i + 1) % 2)
             run_set(i % 2)
+        join_exchange()
         stream.wait_event(freed[(n - 1) % 2])     # the last read-back is inside the region
 
     e2e_steps(args.warmup)
@@ -600,8 +627,9 @@ def run_ours(args):
     bwd_tflops = 6.0 * T * H * V / (bwd_ms * 1e-3) / 1e12
     t4_tflops = flops_tok * T4 / (t4_ms * 1e-3) / 1e12
     q_tflops = 2.0 * T4 * H * V / (q_ms * 1e-3) / 1e12
-    launches_per_step = 3 + (1 if use_rs else 0)   # fwd pair kernel, combine, bwd pair
-                                                    # kernel (+ the ordered sum of dW)
+    # fwd pair kernel, combine, bwd pair kernel (+ the ordered sums of dW: one
+    # per chunk group when overlapped, one otherwise)
+    launches_per_step = 3 + ((groups if overlap else 1) if use_rs else 0)
     value = tokens_all / (ms_max * 1e-3)
     line = {
         "metric": METRIC,
@@ -670,6 +698,8 @@ def run_ours(args):
         "dw_exchange": {"included": bool(use_rs),
                         "kind": "deterministic reduce-scatter of dW: NCCL all-to-all of "
                                 "vocab-row slices, then the rank-ordered sum (rlk_sum_ordered)",
+                        "overlapped": bool(overlap),
+                        "groups": int(groups) if overlap else (1 if use_rs else 0),
                         "bytes_sent_per_rank": (int((world - 1) * -(-V // world) * H * 4)
                                                 if use_rs else 0)},
         "decode_fwd": decode,
@@ -754,6 +784,11 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=48)
     ap.add_argument("--ref-rows", type=int, default=48,
                     help="rows of the RL step the reference arm (the fp64 oracle) runs per step")
+    ap.add_argument("--dw-exchange", choices=["overlap", "after"], default="overlap",
+                    help="N > 1: overlap the dW exchange with the backward (chunk groups on a "
+                         "second stream) or run it after the backward")
+    ap.add_argument("--dw-group-chunks", type=int, default=4,
+                    help="vocab chunks per group of the overlapped dW exchange")
     ap.add_argument("--no-dw-reduce", action="store_true",
                     help="N > 1: leave out the deterministic dW reduce-scatter from the step")
     ap.add_argument("--profile", choices=["fwd", "bwd", "transition", "cublas"], default=None,

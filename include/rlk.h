@@ -287,6 +287,35 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
                              int64_t K, int a_mn_major, int b_mn_major, float* C,
                              void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward that publishes each vocab chunk's completion, so that the
+ * data-parallel exchange of dW (the one exchange of a token-sharded step; the
+ * pages' deterministic collectives: VIME Qwen3-8B TP4/CP2 page, "Required
+ * gates") can start on a chunk's rows while later chunks still compute.
+ * Arguments, layouts, results and errors are those of rlk_linear_logp_bwd,
+ * plus: chunk_done, a caller-owned device array of
+ * ceil(V / rlk_bwd_chunk_width(V)) 32-bit words, and seq >= 1.  Chunk c
+ * covers W rows [c * width, (c + 1) * width); its word is set to seq (a
+ * system-scope release store) once its dW rows (and its dHidden terms) are
+ * written.  Give every call a larger seq than the last one on the same words
+ * (the words are never cleared).  After a timed-out internal wait every word
+ * is set to seq as well, so waiters are released; rlk_read_device_error then
+ * reports RLK_DEVERR_TIMEOUT and the results are not to be used.  T = 0:
+ * dW is zeroed and the words set in stream order.  chunk_done null or
+ * seq = 0: RLK_ERR_INVALID_ARG. */
+rlk_status rlk_linear_logp_bwd_signal(const rlk_bf16* hidden, const rlk_bf16* W,
+                                      const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                      float temperature, const float* lse, const float* entropy,
+                                      const float* dlogp, const float* dentropy,
+                                      rlk_bf16* dHidden, float* dW, void* workspace,
+                                      size_t workspace_bytes, uint32_t* chunk_done, uint32_t seq,
+                                      void* stream);
+
+/* Makes `stream` wait (on the device, no host sync) until *chunk_word >= seq:
+ * a stream memory wait on a word rlk_linear_logp_bwd_signal publishes.  Work
+ * enqueued on `stream` afterwards sees the chunk's dW rows.  chunk_word
+ * device memory, 4-byte aligned; seq >= 1. */
+rlk_status rlk_stream_wait_chunk(const uint32_t* chunk_word, uint32_t seq, void* stream);
+
 /* Fixed-order sum out[i] = ((parts[0][i] + parts[1][i]) + parts[2][i]) + ...
  * over nparts (1..64) equally sized fp32 device buffers of `count` elements;
  * `parts` is a HOST array of device pointers.  The data-parallel exchange of

@@ -159,6 +159,49 @@ def rlk_linear_logp_bwd(hidden, W, targets, temperature, lse, entropy, dlogp, de
     return dHidden, dW
 
 
+_signal_fns = None
+
+
+def _signal():
+    global _signal_fns
+    if _signal_fns is None:
+        L = lib()
+        f = L.rlk_linear_logp_bwd_signal
+        f.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, _P, _P,
+                      ctypes.c_size_t, _P, ctypes.c_uint32, _P]
+        f.restype = ctypes.c_int
+        w = L.rlk_stream_wait_chunk
+        w.argtypes = [_P, ctypes.c_uint32, _P]
+        w.restype = ctypes.c_int
+        _signal_fns = (f, w)
+    return _signal_fns
+
+
+def rlk_linear_logp_bwd_signal(hidden, W, targets, temperature, lse, entropy, dlogp, dentropy,
+                               workspace, out, chunk_done, seq, stream=None):
+    """rlk_linear_logp_bwd that also sets chunk_done[c] (int32 device words, one
+    per vocab chunk of rlk_bwd_chunk_width(V) rows) to seq once chunk c's dW
+    rows are written."""
+    T, H = hidden.shape
+    V = W.shape[0]
+    dHidden, dW = out
+    if chunk_done.dtype != torch.int32 or not chunk_done.is_cuda or \
+            chunk_done.numel() < -(-V // bwd_chunk_width(V)):
+        raise ValueError("chunk_done: int32 CUDA tensor with one word per vocab chunk")
+    _check(_signal()[0](_ptr(hidden), _ptr(W), _ptr(targets), T, H, V, float(temperature),
+                        _ptr(lse), _ptr(entropy), _ptr(dlogp), _ptr(dentropy), _ptr(dHidden),
+                        _ptr(dW), _ptr(workspace), workspace.numel(), _ptr(chunk_done), int(seq),
+                        _stream(stream)),
+           "rlk_linear_logp_bwd_signal")
+    return dHidden, dW
+
+
+def rlk_stream_wait_chunk(chunk_word, seq, stream=None):
+    """Makes `stream` wait on the device until chunk_word (a one-element int32
+    CUDA tensor view) holds seq or more."""
+    _check(_signal()[1](_ptr(chunk_word), int(seq), _stream(stream)), "rlk_stream_wait_chunk")
+
+
 _stall_fn = None
 
 

@@ -189,6 +189,21 @@ bool map_mnmajor(CUtensorMap* m, const void* base, int64_t MN, int64_t K, int64_
   return make_map(m, base, MN, K, pitch, 64, 64);
 }
 
+typedef CUresult (*StreamWaitValueFn)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+typedef CUresult (*StreamWriteValueFn)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+
+// Sets n chunk-completion words to `seq` in stream order (no kernel).
+rlk_status write_chunk_words(uint32_t* words, int64_t n, uint32_t seq, cudaStream_t st) {
+  static const StreamWriteValueFn write =
+      reinterpret_cast<StreamWriteValueFn>(driver_fn("cuStreamWriteValue32"));
+  if (!write) return RLK_ERR_CUDA;
+  for (int64_t c = 0; c < n; ++c)
+    if (write(static_cast<CUstream>(st), reinterpret_cast<CUdeviceptr>(words + c), seq, 0) !=
+        CUDA_SUCCESS)
+      return RLK_ERR_CUDA;
+  return RLK_OK;
+}
+
 std::atomic<int> g_max_clusters[3][kMaxDevices];
 
 // Launches pair_kernel<Mode> on clusters of two CTAs: at most one cluster per
@@ -387,7 +402,8 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
                        const float* dlogp, const float* dentropy, rlk_bf16* dHidden,
                        float* dh_parts, int64_t part_rows, int64_t part_chunks, float* dW,
                        uint8_t* ws, const Layout& L, cudaStream_t st,
-                       uint64_t wait_limit_ns = kWaitLimitNs, int stall_first_h = 0) {
+                       uint64_t wait_limit_ns = kWaitLimitNs, int stall_first_h = 0,
+                       uint32_t* chunk_done = nullptr, uint32_t seq = 0) {
   BwdParams P;
   P.plan = make_bwd_plan(T, H, Vloc, vchunk(Vfull));
   const BwdPlan& pl = P.plan;
@@ -439,6 +455,8 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   P.inv_tau = 1.0f / temperature;
   P.wait_limit_ns = wait_limit_ns;
   P.stall_first_h = stall_first_h;
+  P.chunk_done = chunk_done;
+  P.seq = seq;
 
   if (cudaMemsetAsync(cnt, 0, bwd_counter_words(pl) * 4, st) != cudaSuccess) return RLK_ERR_CUDA;
   // Units wait on units claimed earlier, and only running CTA pairs claim
@@ -552,6 +570,63 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
   return enqueue_bwd(hidden, W, targets, T, H, V, 0, V, temperature, lse, entropy, dlogp,
                      dentropy, dHidden, nullptr, 0, 0, dW, static_cast<uint8_t*>(workspace), L,
                      static_cast<cudaStream_t>(stream), wait_limit_ns, stall != 0 ? 1 : 0);
+}
+
+// The backward that publishes each vocab chunk's completion (declared in
+// rlk.h with the exchange it serves).
+rlk_status rlk_linear_logp_bwd_signal(const rlk_bf16* hidden, const rlk_bf16* W,
+                                      const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                      float temperature, const float* lse, const float* entropy,
+                                      const float* dlogp, const float* dentropy,
+                                      rlk_bf16* dHidden, float* dW, void* workspace,
+                                      size_t workspace_bytes, uint32_t* chunk_done, uint32_t seq,
+                                      void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (!chunk_done || seq == 0) return RLK_ERR_INVALID_ARG;
+  if (!aligned(chunk_done, 4)) return RLK_ERR_MISALIGNED;
+  if (T == 0) {
+    // nothing to compute: dW is zero and every chunk is complete at once
+    if ((s = rlk_linear_logp_bwd(hidden, W, targets, T, H, V, temperature, lse, entropy, dlogp,
+                                 dentropy, dHidden, dW, workspace, workspace_bytes, stream)) !=
+        RLK_OK)
+      return s;
+    return write_chunk_words(chunk_done, ceil_div(V, vchunk(V)), seq,
+                             static_cast<cudaStream_t>(stream));
+  }
+  if (!dW || !hidden || !W || !targets || !lse || !entropy || !dlogp || !dentropy || !dHidden ||
+      !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(dHidden, 16) || !aligned(dW, 16) ||
+      !aligned(workspace, 256) || !aligned(targets, 8) || !aligned(lse, 4) ||
+      !aligned(entropy, 4) || !aligned(dlogp, 4) || !aligned(dentropy, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);
+  if (workspace_bytes < L.bwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  if ((s = enqueue_bwd(hidden, W, targets, T, H, V, 0, V, temperature, lse, entropy, dlogp,
+                       dentropy, dHidden, nullptr, 0, 0, dW, static_cast<uint8_t*>(workspace), L,
+                       static_cast<cudaStream_t>(stream), kWaitLimitNs, 0, chunk_done, seq)) !=
+      RLK_OK)
+    return s;
+  g_calls[1].fetch_add(1);
+  return RLK_OK;
+}
+
+rlk_status rlk_stream_wait_chunk(const uint32_t* chunk_word, uint32_t seq, void* stream) {
+  if (!chunk_word || seq == 0) return RLK_ERR_INVALID_ARG;
+  if (!aligned(chunk_word, 4)) return RLK_ERR_MISALIGNED;
+  int sms = 0;
+  rlk_status s = check_device(&sms);
+  if (s != RLK_OK) return s;
+  static const StreamWaitValueFn wait =
+      reinterpret_cast<StreamWaitValueFn>(driver_fn("cuStreamWaitValue32"));
+  if (!wait) return RLK_ERR_CUDA;
+  return wait(static_cast<CUstream>(stream), reinterpret_cast<CUdeviceptr>(chunk_word), seq,
+              CU_STREAM_WAIT_VALUE_GEQ) == CUDA_SUCCESS
+             ? RLK_OK
+             : RLK_ERR_CUDA;
 }
 
 size_t rlk_gemm_workspace_bytes(void) { return kHeader; }

@@ -82,6 +82,9 @@ struct BwdParams {
   int mn3;            // w_mn, hid_mn, dx_mn are 3-D maps (one box per 128 MN columns)
   uint64_t wait_limit_ns;  // bound of every wait (kWaitLimitNs outside the test hook)
   int stall_first_h;  // test hook: the first dHidden unit waits for one R unit too many
+  uint32_t* chunk_done;  // null, or [NC] words: chunk c's word is set to `seq` once its
+                         // dHidden and dW units are done (for an exchange that overlaps)
+  uint32_t seq;
 };
 
 enum : int { kUnitR = 0, kUnitH = 1, kUnitD = 2 };

@@ -601,11 +601,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (j.type == kUnitR) {
               atomicAdd(P.rdone_m + static_cast<size_t>(j.c) * pl.MT + j.mt, 1u);
               atomicAdd(P.rdone_j + static_cast<size_t>(j.c) * pl.RT_full + j.nt, 1u);
-            } else if (j.type == kUnitH) {
-              atomicAdd(P.hdone + (static_cast<size_t>(j.c) * pl.MT + j.mt) * pl.NH + j.nt, 1u);
-              atomicAdd(P.bufdone + j.c, 1u);
             } else {
-              atomicAdd(P.bufdone + j.c, 1u);
+              if (j.type == kUnitH)
+                atomicAdd(P.hdone + (static_cast<size_t>(j.c) * pl.MT + j.mt) * pl.NH + j.nt,
+                          1u);
+              const uint32_t done = atomicAdd(P.bufdone + j.c, 1u) + 1u;
+              // the CTA that completes chunk c's dHidden and dW units publishes
+              // it: every other CTA's stores were fenced before its increment
+              if (P.chunk_done != nullptr &&
+                  done == 2u * static_cast<uint32_t>(bwd_nH(pl) + bwd_nD(pl, j.c))) {
+                __threadfence_system();
+                st_release_sys_u32(P.chunk_done + j.c, P.seq);
+              }
             }
           }
         }
@@ -618,6 +625,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (Mode == kModeBwd) {
+    // After a timed-out wait some chunks never complete: publish every chunk
+    // word anyway, so that a stream waiting on them is released (the error
+    // word already says the results are not to be used).
+    if (*abort_flag && threadIdx.x == 0 && P.chunk_done != nullptr) {
+      __threadfence_system();
+      for (int c = 0; c < P.plan.NC; ++c) st_release_sys_u32(P.chunk_done + c, P.seq);
+    }
+  }
   if (*abort_flag) {
     // Unwind after a timed-out wait: let TMA loads and MMAs in flight finish
     // before the shared memory and TMEM they touch go away.

@@ -223,6 +223,12 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
+// Store with release semantics at system scope (a word another stream's
+// memory wait, or the host, observes).
+__device__ __forceinline__ void st_release_sys_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Orders this thread's generic-proxy global accesses with its later (or
 // earlier) async-proxy ones, e.g. a TMA load of data another CTA stored.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -278,3 +278,51 @@ def test_tp_autograd_wrapper_plumbing():
         # backward receives the saved lse / entropy and the upstream gradients
         assert calls[1] == ("bwd", 3.0, 2.0, 0.5, 0.25)
         assert dh == 5.0 and wshape == [11 + r, H] and dw == 7.0 and lp0 == -1.0 - r
+
+
+def _rs_overlap_worker(rank, world, port, V, H, chunk, gc, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from invariant_lm_head_gemm_b200 import dp
+    waited = []
+    res, pieces = dp.reduce_scatter_dw_overlapped(
+        _dw(rank, V, H), chunk, chunk_done=list(range(100)), seq=7, group_chunks=gc,
+        sum_fn=_cpu_ordered_sum, wait_fn=lambda word, seq, stream: waited.append((word, seq)))
+    out[rank] = (pieces, res.numpy().tobytes(), waited)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world,V,chunk,gc", [(2, 37, 8, 2), (3, 70, 16, 1), (2, 5, 8, 4),
+                                              (3, 100, 8, 3)])
+def test_overlapped_dw_exchange_is_the_rank_ordered_sum(world, V, chunk, gc):
+    """The chunk-group exchange: every rank's pieces hold the rank-ordered sum
+    of those rows bit for bit, the pieces of all ranks cover [0, V) once, and
+    each group waits for every one of its chunks (in order) before it moves."""
+    H = 4
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rs_overlap_worker, args=(world, _free_port(), V, H, chunk, gc, out),
+                 nprocs=world, join=True)
+        res = dict(out)
+    full = _dw(0, V, H)
+    for r in range(1, world):
+        full = full + _dw(r, V, H)          # rank order
+    seen = np.zeros(V, dtype=int)
+    nchunks = -(-V // chunk)
+    for r in range(world):
+        pieces, raw, waited = res[r]
+        got = np.frombuffer(raw, dtype=np.float32).reshape(-1, H)
+        off = 0
+        for r0, r1 in pieces:
+            assert np.array_equal(got[off:off + r1 - r0].view(np.uint32),
+                                  full[r0:r1].numpy().view(np.uint32))
+            seen[r0:r1] += 1
+            off += r1 - r0
+        assert waited == [([c], 7) for c in range(nchunks)]
+    assert (seen == 1).all()
