@@ -348,10 +348,12 @@ rlk_status rlk_read_device_error(void* workspace, uint32_t* flags, void* stream)
  * workspace's error word, lets its in-flight copies and MMAs finish, frees its
  * tensor memory and returns, and the outputs are not to be used.
  * rlk_test_linear_logp_bwd_stall is rlk_linear_logp_bwd (same arguments,
- * layouts and ownership) with two more: wait_limit_ns bounds every wait of the
- * launch (1 ms .. 2 s; the production entry points use 2 s), and stall != 0
+ * layouts and ownership) with more: wait_limit_ns bounds every wait of the
+ * launch (1 ms .. 2 s; the production entry points use 2 s); stall != 0
  * makes the first dHidden unit wait for one more recompute tile than exists,
- * a dependency nothing ever meets.  With stall set the call still returns
+ * a dependency nothing ever meets; chunk_done / seq, when chunk_done is not
+ * null, publish vocab-chunk completion as rlk_linear_logp_bwd_signal does
+ * (so the release of the words after a timeout can be tested).  With stall set the call still returns
  * RLK_OK (the launch is enqueued); rlk_read_device_error then reports
  * RLK_DEVERR_TIMEOUT, and later calls on the same workspace and stream behave
  * as on a fresh one.  T = 0 or a limit outside the range: RLK_ERR_INVALID_ARG. */
@@ -361,7 +363,8 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
                                           const float* entropy, const float* dlogp,
                                           const float* dentropy, rlk_bf16* dHidden, float* dW,
                                           void* workspace, size_t workspace_bytes,
-                                          uint64_t wait_limit_ns, int stall, void* stream);
+                                          uint64_t wait_limit_ns, int stall,
+                                          uint32_t* chunk_done, uint32_t seq, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* rlk_status_string(rlk_status status);

@@ -207,7 +207,7 @@ _stall_fn = None
 
 def rlk_test_linear_logp_bwd_stall(hidden, W, targets, temperature, lse, entropy, dlogp,
                                    dentropy, workspace, out, wait_limit_ns, stall,
-                                   stream=None):
+                                   chunk_done=None, seq=0, stream=None):
     """Test hook of the fail-closed path: the backward with every wait bounded
     by wait_limit_ns and, when stall is set, one dependency that is never met
     (the device error word then reports RLK_DEVERR_TIMEOUT)."""
@@ -215,7 +215,7 @@ def rlk_test_linear_logp_bwd_stall(hidden, W, targets, temperature, lse, entropy
     if _stall_fn is None:
         f = lib().rlk_test_linear_logp_bwd_stall
         f.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _P, _P, _P, _P,
-                      ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, _P]
+                      ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, _P, ctypes.c_uint32, _P]
         f.restype = ctypes.c_int
         _stall_fn = f
     T, H = hidden.shape
@@ -224,7 +224,7 @@ def rlk_test_linear_logp_bwd_stall(hidden, W, targets, temperature, lse, entropy
     _check(_stall_fn(_ptr(hidden), _ptr(W), _ptr(targets), T, H, V, float(temperature), _ptr(lse),
                      _ptr(entropy), _ptr(dlogp), _ptr(dentropy), _ptr(dHidden), _ptr(dW),
                      _ptr(workspace), workspace.numel(), int(wait_limit_ns), int(stall),
-                     _stream(stream)),
+                     _ptr(chunk_done), int(seq), _stream(stream)),
            "rlk_test_linear_logp_bwd_stall")
     return dHidden, dW
 

@@ -551,11 +551,13 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
                                           const float* entropy, const float* dlogp,
                                           const float* dentropy, rlk_bf16* dHidden, float* dW,
                                           void* workspace, size_t workspace_bytes,
-                                          uint64_t wait_limit_ns, int stall, void* stream) {
+                                          uint64_t wait_limit_ns, int stall,
+                                          uint32_t* chunk_done, uint32_t seq, void* stream) {
   rlk_status s = check_sizes(T, H, V, temperature);
   if (s != RLK_OK) return s;
   if (T == 0 || wait_limit_ns < 1000000ull || wait_limit_ns > kWaitLimitNs)
     return RLK_ERR_INVALID_ARG;  // 1 ms .. 2 s
+  if (chunk_done != nullptr && (seq == 0 || !aligned(chunk_done, 4))) return RLK_ERR_INVALID_ARG;
   if (!hidden || !W || !targets || !lse || !entropy || !dlogp || !dentropy || !dHidden || !dW ||
       !workspace)
     return RLK_ERR_INVALID_ARG;
@@ -569,7 +571,8 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
   if ((s = check_device(&sms)) != RLK_OK) return s;
   return enqueue_bwd(hidden, W, targets, T, H, V, 0, V, temperature, lse, entropy, dlogp,
                      dentropy, dHidden, nullptr, 0, 0, dW, static_cast<uint8_t*>(workspace), L,
-                     static_cast<cudaStream_t>(stream), wait_limit_ns, stall != 0 ? 1 : 0);
+                     static_cast<cudaStream_t>(stream), wait_limit_ns, stall != 0 ? 1 : 0,
+                     chunk_done, seq);
 }
 
 // The backward that publishes each vocab chunk's completion (declared in

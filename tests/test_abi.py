@@ -234,11 +234,13 @@ def test_stall_hook_rejects_limits_outside_its_range(L):
     anything touches the device: these pointers are never dereferenced."""
     f = L.rlk_test_linear_logp_bwd_stall
     f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_float] + \
-        [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+        [ctypes.c_void_p] * 7 + [ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int,
+                                 ctypes.c_void_p, ctypes.c_uint32, ctypes.c_void_p]
     f.restype = ctypes.c_int
     p = 0x10000
     args = [p, p, p, 4, 64, 100, 1.0, p, p, p, p, p, p, p, 1 << 20]
-    assert f(*args, 10, 1, None) == INVALID               # below 1 ms
-    assert f(*args, 3_000_000_000, 1, None) == INVALID    # above 2 s
+    assert f(*args, 10, 1, None, 0, None) == INVALID               # below 1 ms
+    assert f(*args, 3_000_000_000, 1, None, 0, None) == INVALID    # above 2 s
     assert f(p, p, p, 0, 64, 100, 1.0, p, p, p, p, p, p, p, 1 << 20, 100_000_000, 1,
-             None) == INVALID                              # T = 0
+             None, 0, None) == INVALID                              # T = 0
+    assert f(*args, 100_000_000, 1, p, 0, None) == INVALID         # words without seq

@@ -46,14 +46,24 @@ def test_stalled_backward_reports_timeout_and_the_next_call_is_unaffected():
     assert binding.rlk_read_device_error(ws) == 0
     assert torch.equal(_bits(out[0]), _bits(dH_ref)) and torch.equal(_bits(out[1]), _bits(dW_ref))
 
-    # a dependency nothing meets: the call returns, the error word says timeout
+    # a dependency nothing meets: the call returns, the error word says timeout,
+    # and every vocab-chunk completion word is published anyway, so a stream
+    # waiting on them (an overlapped dW exchange) is released
+    nchunks = -(-V // binding.bwd_chunk_width(V))
+    words = torch.zeros(nchunks, dtype=torch.int32, device="cuda")
     t0 = time.perf_counter()
-    binding.rlk_test_linear_logp_bwd_stall(hid, W, tg, tau, ls, en, dl, de, ws, out, LIMIT_NS, 1)
+    binding.rlk_test_linear_logp_bwd_stall(hid, W, tg, tau, ls, en, dl, de, ws, out, LIMIT_NS, 1,
+                                           chunk_done=words, seq=5)
     torch.cuda.synchronize()
     elapsed = time.perf_counter() - t0
     flags = binding.rlk_read_device_error(ws)
     assert flags & binding.RLK_DEVERR_TIMEOUT, flags
     assert elapsed < 60.0, elapsed
+    assert (words == 5).all()
+    side = torch.cuda.Stream()
+    for c in range(nchunks):
+        binding.rlk_stream_wait_chunk(words[c:c + 1], 5, side)
+    side.synchronize()
 
     # the next calls on the same workspace and stream are bit for bit those of
     # a fresh run
