@@ -389,14 +389,15 @@ def run_ours(args):
         torch.cuda.synchronize()
         return 1e3 * e_a.elapsed_time(e_b) / 20, eager
 
-    decode_rows = (1, 4, 16, 64, 128, 256)
+    decode_rows = (1, 4, 16, 64, 128, 192, 256)
     for Td in decode_rows:
         decode_us(Td)
     dec_us = [decode_us(Td) for Td in decode_rows]
     dec_gbs = [(V * H * 2 + Td * (H * 2 + 8 + 12)) / (u * 1e-6) / 1e9
                for Td, (u, _) in zip(decode_rows, dec_us)]
-    decode = {"kernel": "decode_fwd_kernel (T <= 128: operands swapped, M = 128 vocab rows, "
-                        "N = T padded to 16/32) + combine; larger T: the pair kernel",
+    decode = {"kernel": "decode_fwd_kernel (T <= 224: operands swapped, 128 vocab rows per CTA, "
+                        "N = T padded to 16/32; single-CTA MMA for N <= 32, CTA-pair MMA "
+                        "(M = 256) from N = 64) + combine; larger T: the pair kernel",
               "bound": "hbm", "unit": "GB/s", "timing": "CUDA-graph replay, 20 calls",
               "rows": list(decode_rows), "us_per_call": [u for u, _ in dec_us],
               "eager_us_per_call": [e for _, e in dec_us], "achieved": dec_gbs,

@@ -264,9 +264,10 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
 // target falls in these rows, the target's scaled logit to ytgt.
 static_assert(kDecSplit == kBN * kFwdGroup, "both forward kernels must use the same splits");
 
-std::atomic<int> g_dec_max_clusters[kDecMaxRows / 16][kMaxDevices];  // by N / 16 - 1
+std::atomic<int> g_dec_max_clusters[2][kDecMaxRows / 16][kMaxDevices];  // by form, N / 16 - 1
 
-// Forward partials for T <= kDecMaxRows (decode_fwd_kernel, rlk_decode.cuh).
+// Forward partials for T <= kDecMaxT (decode_fwd_kernel, rlk_decode.cuh):
+// the single-CTA MMA form below N = kDecPairMinN, the CTA-pair form from there.
 rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
                                       const int64_t* targets, int64_t T, int64_t H, int64_t Vloc,
                                       int64_t v0, float temperature, float* part_m, float* part_s,
@@ -274,7 +275,10 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
                                       cudaStream_t st) {
   DecArgs a;
   a.N = T <= 16 ? 16 : static_cast<int>(ceil_div(T, 32) * 32);
-  if (!map_kmajor(&a.w_k, W, H, Vloc, H, kBM) || !map_kmajor(&a.hid_k, hidden, H, T, H, a.N))
+  const bool pair = a.N >= kDecPairMinN;
+  // the pair form splits the N hidden rows between the two CTAs (N / 2 each)
+  if (!map_kmajor(&a.w_k, W, H, Vloc, H, kBM) ||
+      !map_kmajor(&a.hid_k, hidden, H, T, H, pair ? a.N / 2 : a.N))
     return RLK_ERR_CUDA;
   a.ep.targets = targets;
   a.ep.part_m = part_m;
@@ -290,16 +294,17 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
   a.KB = static_cast<int>(H / kBK);
   a.NG = static_cast<int>(fwd_groups(Vloc));
   constexpr uint32_t kSmemLimit = 227u * 1024u;
-  a.stages = kDecMaxStages;
-  while (a.stages > 2 && dec_smem_bytes(a.N, a.stages) > kSmemLimit) --a.stages;
-  const uint32_t smem = dec_smem_bytes(a.N, a.stages);
+  a.stages = dec_stages(a.N, pair, kSmemLimit);
+  if (a.stages == 0) return RLK_ERR_CUDA;
+  const uint32_t smem = dec_smem_bytes(a.N, a.stages, pair);
+  void (*kern)(DecArgs) = pair ? decode_fwd_kernel<true> : decode_fwd_kernel<false>;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return RLK_ERR_CUDA;
   }
-  if (cudaFuncSetAttribute(decode_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemLimit)) != cudaSuccess) {
     cudaGetLastError();
     return RLK_ERR_CUDA;
@@ -315,19 +320,20 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int mc = g_dec_max_clusters[a.N / 16 - 1][dev].load(std::memory_order_relaxed);
+  std::atomic<int>& cache = g_dec_max_clusters[pair ? 1 : 0][a.N / 16 - 1][dev];
+  int mc = cache.load(std::memory_order_relaxed);
   if (mc == 0) {
     cfg.gridDim = dim3(kDecCluster);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_fwd_kernel, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
       cudaGetLastError();
       return RLK_ERR_CUDA;
     }
     mc = n;
-    g_dec_max_clusters[a.N / 16 - 1][dev].store(n, std::memory_order_relaxed);
+    cache.store(n, std::memory_order_relaxed);
   }
   cfg.gridDim = dim3(static_cast<unsigned>(kDecCluster * std::min<int>(a.NG, mc)));
-  if (cudaLaunchKernelEx(&cfg, decode_fwd_kernel, a) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, a) != cudaSuccess) {
     cudaGetLastError();
     return RLK_ERR_CUDA;
   }
@@ -338,7 +344,7 @@ rlk_status enqueue_fwd_partials(const rlk_bf16* hidden, const rlk_bf16* W, const
                                 int64_t T, int64_t H, int64_t Vloc, int64_t v0, float temperature,
                                 float* part_m, float* part_s, float* part_b, int64_t ldp,
                                 float* ytgt, uint32_t* err, cudaStream_t st) {
-  if (T <= kDecMaxRows)
+  if (T <= kDecMaxT)
     return enqueue_fwd_partials_short(hidden, W, targets, T, H, Vloc, v0, temperature, part_m,
                                       part_s, part_b, ldp, ytgt, err, st);
   FwdArgs a;

@@ -1,4 +1,4 @@
-// rlk_decode.cuh -- forward for short batches (rollout / decode shapes, T <= 128
+// rlk_decode.cuh -- forward for short batches (rollout / decode shapes, T <= 224
 // rows): the same per-split triples as the pair kernel's forward, produced
 // with the operands swapped so that the tensor cores do not pad T up to 256.
 //
@@ -12,10 +12,23 @@
 // of W (one K block per stage held the stages ~20% longer for the same
 // bytes).
 //
+// Two forms of the MMA, chosen by N:
+//  * single (kPair = false, N < 64): tcgen05.mma.cta_group::1, M = 128; each
+//    CTA holds its 128 W rows and all N hidden rows per K block;
+//  * pair (kPair = true, 64 <= N <= 256): tcgen05.mma.cta_group::2, M = 256
+//    over CTAs (2i, 2i+1) of the cluster; each CTA still holds its own 128 W
+//    rows but only half of the N hidden rows (B is split along N across the
+//    pair), and each CTA's TMEM receives its 128 W rows x all N columns, so
+//    the epilogue is the same.  Halving the hidden bytes per CTA leaves room
+//    for more stages of W in flight (N = 128: four instead of three) and lets
+//    N reach 256 (three stages), where the single form would hold 64 KB of
+//    hidden per stage.
+//
 // Numerics are those of the pair kernel, bit for bit:
 //  * each logit is the same bf16 dot product over H in the same 64-wide K
 //    blocks and 16-wide MMA steps (D = A . B^T gives the same fp32 element
-//    with A and B exchanged: each element is its own product sum);
+//    with A and B exchanged and whatever the M / N shape: each element is its
+//    own product sum);
 //  * a vocab split is 512 columns = four 128-row W tiles, one per CTA of a
 //    cluster of four.  CTA r runs the split's chunks r*4 .. r*4+3 with
 //    fwd_chunk_update after receiving the running (m, s, b) of every row from
@@ -25,27 +38,55 @@
 //  * CTA 3 writes the split's triple where the pair kernel's forward writes
 //    it, and the same combine kernel merges the splits.
 //
-// Warp roles per CTA (192 threads): warp 0 producer (TMA), warp 1 MMA issuer,
-// warps 2-5 epilogue.  Two TMEM accumulators of up to 128 columns; the
-// epilogue copies an accumulator to shared memory transposed (row-major per
-// batch row), 32 rows at a time, and frees it after the last block.
+// Warp roles per CTA (192 threads): warp 0 producer (TMA), warp 1 MMA issuer
+// (in the pair form only the even CTA of each pair issues), warps 2-5
+// epilogue.  Two TMEM accumulators of up to 128 (single) or 256 (pair)
+// columns.  The epilogue is a pipeline over 32-row batch blocks: the warp
+// that reads TMEM lane quarter q holds chunk q of the tile, transposes its
+// 32 x 32 block through its own shared-memory tile so that each lane holds one
+// batch row, folds that chunk and hands the row's (m, s, b) to the warp of
+// chunk q+1; the warp of chunk 3 hands it on to CTA rank+1 block by block.
+// So the four warps and the four CTAs of a split work on different blocks at
+// once, while each row still folds its 16 chunks in ascending order.  With a
+// single block (N <= 32) there is nothing to overlap: warp 2 folds all four
+// chunks from the four warps' tiles, which keeps the chain of CTAs at one
+// hand-off per CTA.
 #pragma once
 
 #include "rlk_gemm.cuh"
 
 namespace rlk {
 
-constexpr int kDecMaxRows = 128;    // largest T this path takes
+constexpr int kDecMaxRows = 256;    // largest N of the pair form (hand buffer rows)
+constexpr int kDecMaxT = 224;       // largest T the launcher sends here: at N = 256 a stage
+                                    // holds as much hidden as W and the pair kernel is faster
+constexpr int kDecSingleMaxN = 128; // largest N of the single form
+constexpr int kDecPairMinN = 64;    // N from which the pair form is launched
 constexpr int kDecCluster = 4;      // CTAs per vocab split
 constexpr int kDecThreads = 192;
 constexpr int kDecMaxStages = 12;
-constexpr int kDecYStride = 132;    // floats per batch row of the transposed tile
-constexpr int kDecTmemCols = 256;   // two accumulators of up to 128 columns
+constexpr int kDecXStride = 33;     // floats per row of a warp's 32 x 32 transposition tile
+constexpr int kDecYStride = 132;    // floats per batch row of the one-block tile (same memory)
+static_assert(32 * kDecYStride == 4 * 32 * kDecXStride, "the one-block tile reuses the four tiles");
+constexpr int kDecMaxBlocks = kDecMaxRows / 32;  // 32-row batch blocks of the widest N
 constexpr int kDecSplit = kDecCluster * kBM;
 constexpr int kDecKPerStage = 2;   // K blocks per pipeline stage
 constexpr uint32_t kDecABox = kBM * kBK * 2;                    // one 128 x 64 W box
 constexpr uint32_t kDecABytes = kDecKPerStage * kDecABox;       // a stage's W boxes
-constexpr int kDecNumBars = 2 * kDecMaxStages + 9;
+// full, empty per stage; tfull, tempty per accumulator; hfull per (hand
+// buffer, block), hempty per hand buffer; pfull, pempty per warp link; xfull,
+// xfree of the one-block epilogue; drain
+constexpr int kDecNumBars = 2 * kDecMaxStages + 4 + 2 * kDecMaxBlocks + 2 + 6 + 2 + 1;
+// floats of the epilogue's shared memory besides the hand buffers: four 32 x 33
+// transposition tiles and three (m, s, b) x 32 links between the warps
+constexpr uint32_t kDecEpiFloats = 4u * 32u * kDecXStride + 3u * 3u * 32u;
+
+// Batch rows (and TMEM columns per accumulator) of each form.
+template <bool kPair>
+struct DecForm {
+  static constexpr int kMaxRows = kPair ? kDecMaxRows : kDecSingleMaxN;
+  static constexpr uint32_t kTmemCols = 2u * kMaxRows;  // two accumulators (a power of 2)
+};
 
 struct DecArgs {
   CUtensorMap w_k;    // W [V, H], K-major, box 64 x 128
@@ -53,47 +94,77 @@ struct DecArgs {
   EpiFwd::Params ep;  // outputs and layout of the pair kernel's forward
   uint32_t* err;
   int N;              // MMA N: 16 for T <= 16, else T rounded up to 32
+                      // (the hidden box holds N rows, or N / 2 in the pair form)
   int KB;             // H / 64
   int NG;             // vocab splits of this W
   int stages;
 };
 
 // Dynamic shared memory of the kernel for MMA width N and `stages` stages.
-__host__ __device__ constexpr uint32_t dec_smem_bytes(int N, int stages) {
-  return 1024u + static_cast<uint32_t>(stages) * (kDecABytes + N * kBK * 2u * kDecKPerStage) +
-         32u * kDecYStride * 4u + 2u * 3u * kDecMaxRows * 4u +
+__host__ __device__ constexpr uint32_t dec_smem_bytes(int N, int stages, bool pair) {
+  return 1024u +
+         static_cast<uint32_t>(stages) *
+             (kDecABytes + static_cast<uint32_t>(pair ? N / 2 : N) * kBK * 2u * kDecKPerStage) +
+         kDecEpiFloats * 4u + 2u * 3u * static_cast<uint32_t>(pair ? kDecMaxRows : kDecSingleMaxN) * 4u +
          kDecNumBars * 8u + 32u;
 }
 
+// The stage count the launcher takes for MMA width N: the most, at most
+// kDecMaxStages, whose plan fits in `limit` bytes; 0 if two stages do not fit.
+__host__ __device__ constexpr int dec_stages(int N, bool pair, uint32_t limit) {
+  int S = kDecMaxStages;
+  while (S >= 2 && dec_smem_bytes(N, S, pair) > limit) --S;
+  return S >= 2 ? S : 0;
+}
+
+template <bool kPair>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid_constant__ DecArgs P) {
+  constexpr int MR = DecForm<kPair>::kMaxRows;  // batch rows a hand buffer holds
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const int N = P.N, S = P.stages;
-  const uint32_t b_box = static_cast<uint32_t>(N) * kBK * 2u;   // one N x 64 hidden box
+  const int NB = kPair ? N / 2 : N;                              // hidden rows this CTA holds
+  const uint32_t b_box = static_cast<uint32_t>(NB) * kBK * 2u;   // one NB x 64 hidden box
   const uint32_t b_bytes = kDecKPerStage * b_box;
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + S * kDecABytes;
-  float* Y = reinterpret_cast<float*>(smem + S * (kDecABytes + b_bytes));  // [32][kDecYStride]
-  float* hand = Y + 32 * kDecYStride;                // [2][3][kDecMaxRows] incoming (m, s, b)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(hand + 2 * 3 * kDecMaxRows);
+  float* XT = reinterpret_cast<float*>(smem + S * (kDecABytes + b_bytes));  // [4][32][kDecXStride]
+  float* pass = XT + 4 * 32 * kDecXStride;           // [3][3][32] (m, s, b) from warp c to c+1
+  float* hand = pass + 3 * 3 * 32;                   // [2][3][MR] incoming (m, s, b)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(hand + 2 * 3 * MR);
   const uint32_t bar0 = smem_u32(bars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kDecNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* ok1 = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  volatile int* ok3 = reinterpret_cast<volatile int*>(tmem_slot + 4);
 
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kDecMaxStages + s); };
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kDecMaxStages + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kDecMaxStages + 2 + a); };
-  // hfull(h): this CTA's hand buffer h was written by CTA rank-1 (128 arrivals)
-  // hempty(h): CTA rank+1 has read what this CTA wrote into its buffer h
-  auto hfull_bar = [&](int h) { return bar0 + 8u * (2 * kDecMaxStages + 4 + h); };
-  auto hempty_bar = [&](int h) { return bar0 + 8u * (2 * kDecMaxStages + 6 + h); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kDecMaxStages + 8);
+  // hfull(h, blk): rows blk*32 .. +31 of this CTA's hand buffer h were written
+  //                by CTA rank-1 (one arrival per lane of its last-chunk warp)
+  // hempty(h): CTA rank+1 has read every row this CTA wrote into its buffer h
+  //            (one arrival per lane of its first-chunk warp)
+  auto hfull_bar = [&](int h, int blk) {
+    return bar0 + 8u * (2 * kDecMaxStages + 4 + h * kDecMaxBlocks + blk);
+  };
+  auto hempty_bar = [&](int h) { return bar0 + 8u * (2 * kDecMaxStages + 4 + 2 * kDecMaxBlocks + h); };
+  // pfull(c) / pempty(c): the link from the warp of chunk c to that of c+1
+  constexpr int kPBar = 2 * kDecMaxStages + 6 + 2 * kDecMaxBlocks;
+  auto pfull_bar = [&](int c) { return bar0 + 8u * (kPBar + c); };
+  auto pempty_bar = [&](int c) { return bar0 + 8u * (kPBar + 3 + c); };
+  // xfull: the four transposition tiles of a one-block unit are written;
+  // xfree: warp 2 has read them
+  const uint32_t xfull_bar = bar0 + 8u * (kPBar + 6);
+  const uint32_t xfree_bar = bar0 + 8u * (kPBar + 7);
+  const uint32_t drain_bar = bar0 + 8u * (kPBar + 8);
 
   const uint32_t rank = cluster_ctarank();
+  // the pair form: CTA 2i issues the MMAs of the pair (2i, 2i+1) and owns its
+  // full / accumulator-empty barriers; commits arrive in both CTAs
+  const uint32_t lead = kPair ? (rank & ~1u) : rank;
+  const bool is_lead = rank == lead;
+  const uint16_t pair_mask = static_cast<uint16_t>(3u << lead);
   const long long cluster = blockIdx.x / kDecCluster;
   const long long nclusters = gridDim.x / kDecCluster;
   const long long total = P.NG;
@@ -108,17 +179,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);  // one arrival per epilogue warp
-      mbar_init(hfull_bar(a), kDecMaxRows);
-      mbar_init(hempty_bar(a), kDecMaxRows);
+      mbar_init(tempty_bar(a), kPair ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
+      for (int blk = 0; blk < kDecMaxBlocks; ++blk) mbar_init(hfull_bar(a, blk), 32);
+      mbar_init(hempty_bar(a), 32);
     }
+    for (int c = 0; c < 3; ++c) {
+      mbar_init(pfull_bar(c), 32);
+      mbar_init(pempty_bar(c), 32);
+    }
+    mbar_init(xfull_bar, 128);
+    mbar_init(xfree_bar, 32);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kDecTmemCols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), DecForm<kPair>::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), DecForm<kPair>::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -137,12 +219,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
     if (lane == 0) {
       tma_prefetch_desc(&P.w_k);
       tma_prefetch_desc(&P.hid_k);
+      const int h0 = kPair ? static_cast<int>(rank & 1u) * NB : 0;  // first hidden row held here
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
         const long long u = unit_of(k);
         if (u < 0) break;
         const int w0 = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
         const bool a_in = w0 < P.ep.V;  // a tile wholly past V is masked anyway: skip its loads
+        // bytes one K block delivers to the full barrier (both CTAs' in the pair form;
+        // the odd CTA's W tile starts kBM rows after the even one's)
+        uint32_t kb_bytes = (a_in ? kDecABox : 0u) + b_box;
+        if (kPair) kb_bytes += (w0 + kBM < P.ep.V ? kDecABox : 0u) + b_box;
         for (int kb = 0; kb < P.KB; kb += kDecKPerStage) {
           const int nk = min(kDecKPerStage, P.KB - kb);  // K blocks in this stage
           const int s = issued % S;
@@ -151,12 +238,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(s), nk * ((a_in ? kDecABox : 0u) + b_box));
-          for (int i = 0; i < nk; ++i) {
-            if (a_in)
-              tma_load_2d(sA + s * kDecABytes + i * kDecABox, &P.w_k, full_bar(s),
-                          (kb + i) * kBK, w0);
-            tma_load_2d(sB + s * b_bytes + i * b_box, &P.hid_k, full_bar(s), (kb + i) * kBK, 0);
+          if constexpr (kPair) {
+            const uint32_t fb = mapa_shared(full_bar(s), lead);
+            if (is_lead) mbar_arrive_expect_tx(full_bar(s), nk * kb_bytes);
+            for (int i = 0; i < nk; ++i) {
+              if (a_in)
+                tma_load_2d_pair(sA + s * kDecABytes + i * kDecABox, &P.w_k, fb, (kb + i) * kBK, w0);
+              tma_load_2d_pair(sB + s * b_bytes + i * b_box, &P.hid_k, fb, (kb + i) * kBK, h0);
+            }
+          } else {
+            mbar_arrive_expect_tx(full_bar(s), nk * kb_bytes);
+            for (int i = 0; i < nk; ++i) {
+              if (a_in)
+                tma_load_2d(sA + s * kDecABytes + i * kDecABox, &P.w_k, full_bar(s),
+                            (kb + i) * kBK, w0);
+              tma_load_2d(sB + s * b_bytes + i * b_box, &P.hid_k, full_bar(s), (kb + i) * kBK, 0);
+            }
           }
           ++issued;
         }
@@ -165,8 +262,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, N, false, false);
+    if (lane == 0 && is_lead) {
+      const uint32_t idesc = idesc_bf16_f32(kPair ? 2 * kBM : kBM, N, false, false);
       uint32_t it = 0;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
@@ -174,7 +271,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
         const int acc = k & 1;
         if (!mbar_wait_bounded(tempty_bar(acc), ((k >> 1) & 1u) ^ 1u, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kDecMaxRows;
+        const uint32_t d_tmem = tmem_base + acc * MR;
         for (int kb = 0; kb < P.KB; kb += kDecKPerStage, ++it) {
           const int nk = min(kDecKPerStage, P.KB - kb);
           const int s = it % S;
@@ -189,104 +286,236 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t ad = smem_desc_sw128(a_s + i * kDecABox + kk * 32u, 16u, 1024u);
               const uint64_t bd = smem_desc_sw128(b_s + i * b_box + kk * 32u, 16u, 1024u);
-              umma_bf16(d_tmem, ad, bd, idesc, ((kb + i) | kk) != 0 ? 1u : 0u);
+              const uint32_t accum = ((kb + i) | kk) != 0 ? 1u : 0u;
+              if constexpr (kPair) {
+                umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+              } else {
+                umma_bf16(d_tmem, ad, bd, idesc, accum);
+              }
             }
           }
-          umma_commit(empty_bar(s));
+          if constexpr (kPair) {
+            umma_commit_pair_mask(empty_bar(s), pair_mask);
+          } else {
+            umma_commit(empty_bar(s));
+          }
         }
-        if (ok) umma_commit(tfull_bar(acc));
+        if (ok) {
+          if constexpr (kPair) {
+            umma_commit_pair_mask(tfull_bar(acc), pair_mask);
+          } else {
+            umma_commit(tfull_bar(acc));
+          }
+        }
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;              // TMEM lane quarter of this warp
-    const int v_loc = q * 32 + lane;     // W row of the tile held in this thread's lane
-    const int t = (warp - 2) * 32 + lane;  // batch row whose chain this thread runs
-    const bool tvalid = t < P.ep.T;
-    const int64_t tgt = tvalid ? P.ep.targets[t] - P.ep.v0 : -1;
-    const bool ep_leader = threadIdx.x == 64;
+    // Warp q (q = warp & 3) reads TMEM lanes 32q .. 32q+31 = W rows 32q .. +31
+    // of the tile = chunk q of the split's four 32-column chunks in this CTA.
+    // Batch rows flow through the four warps in 32-row blocks: warp q folds
+    // chunk q of a block's rows into their running (m, s, b), which it takes
+    // from warp q-1 (or, for q = 0, from CTA rank-1 / fresh) and hands to warp
+    // q+1 (or, for q = 3, to CTA rank+1 / the split's partial), so every row
+    // still folds its chunks in ascending column order while the four warps
+    // (and the four CTAs) work on different blocks at once.
+    const int q = warp & 3;
+    float* xt = XT + q * 32 * kDecXStride;
+    const int nblk = (N + 31) / 32;
+    // waits of one lane, shared with the warp; then each lane acquires
+    auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_bounded_sleep(bar, parity, abort_flag, err) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) mbar_try_wait(bar, parity);
+      return ok != 0;
+    };
+    auto warp_wait_cluster = [&](uint32_t bar, uint32_t parity) -> bool {
+      int ok = 0;
+      if (lane == 0) ok = mbar_wait_cluster_bounded_sleep(bar, parity, abort_flag, err) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) mbar_try_wait_cluster(bar, parity);
+      return ok != 0;
+    };
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    for (uint32_t k = 0;; ++k) {
+    uint32_t g = 0;  // blocks this warp has passed on (phase of its links)
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
       const long long u = unit_of(k);
       if (u < 0) break;
       const int acc = k & 1, h = k & 1;
       const uint32_t hph = (k >> 1) & 1u;
-      // 1. the accumulator, and the running triple from CTA rank-1 (or a fresh one)
-      if (ep_leader) {
-        bool ok = mbar_wait_bounded(tfull_bar(acc), hph, abort_flag, err);
-        if (ok && rank > 0) ok = mbar_wait_cluster_bounded(hfull_bar(h), hph, abort_flag, err);
-        *ok1 = ok ? 1 : 0;
-      }
-      epilogue_bar();
-      if (!*ok1) break;
+      if (!warp_wait(tfull_bar(acc), hph)) break;
       tc_fence_after();
-      float m = kMaskLogit, s = 0.f, b = 0.f;
-      if (rank > 0) {
-        mbar_try_wait_cluster(hfull_bar(h), hph);  // completed: acquire for this thread
-        const float* in = hand + h * 3 * kDecMaxRows;
-        m = in[t];
-        s = in[kDecMaxRows + t];
-        b = in[2 * kDecMaxRows + t];
-        mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
-      }
-      // 2. 32 batch rows at a time: their accumulator columns go to Y transposed
-      //    (all four warps, one TMEM lane quarter each), then the warp that owns
-      //    those rows folds the tile's four chunks in column order; the
-      //    accumulator is freed after its last columns are read
-      const int col_base = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
-      const int nblk = (N + 31) / 32;
-      for (int blk = 0; blk < nblk; ++blk) {
+      const int tile0 = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
+      const int col0 = tile0 + q * 32;
+      if (nblk == 1) {
+        // One 32-row block (N <= 32): every warp transposes its chunk, then
+        // warp 2 folds all four in order.  Passing the rows from warp to warp
+        // would overlap nothing here and only lengthen the chain of CTAs by
+        // three hand-offs; and warp 2 is the epilogue warp that shares its
+        // scheduler with neither the producer (warp 0) nor the MMA issuer
+        // (warp 1), whose issue latency sets the W stream.
+        // The accumulator is read once the running triples have arrived from
+        // CTA rank-1: releasing it sooner lets the four CTAs of a split drift
+        // apart in their W streams, which measured ~2% slower.  The tile is
+        // row-major per batch row (Y[row][W row of the tile]), in the memory of
+        // the four transposition tiles.
+        const int t = lane;
+        const int64_t tgt = t < P.ep.T ? P.ep.targets[t] - P.ep.v0 : -1;
+        float* Y = XT;
+        if (warp != 2 && k > 0 && !warp_wait(xfree_bar, (k - 1) & 1u)) break;
+        if (rank > 0 && !warp_wait_cluster(hfull_bar(h, 0), hph)) break;
+        const int v_loc = q * 32 + lane;
         if (N == 16) {
           uint32_t r[16];
-          tmem_ld16(tl + acc * kDecMaxRows, r);
+          tmem_ld16(tl + acc * MR, r);
 #pragma unroll
           for (int j = 0; j < 16; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
         } else {
           uint32_t r[32];
-          tmem_ld32(tl + acc * kDecMaxRows + blk * 32, r);
+          tmem_ld32(tl + acc * MR, r);
 #pragma unroll
           for (int j = 0; j < 32; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
         }
-        if (blk == nblk - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(acc));
-        }
-        epilogue_bar();  // Y holds batch rows blk*32 .. +31
-        if (warp - 2 == blk && tvalid) {
-          const float4* row = reinterpret_cast<const float4*>(Y + lane * kDecYStride);
-#pragma unroll 1
-          for (int c = 0; c < kBM / 32; ++c) {
-            float y[32];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 f = row[c * 8 + i];
-              y[4 * i + 0] = fwd_scale(f.x, P.ep.scale_log2);
-              y[4 * i + 1] = fwd_scale(f.y, P.ep.scale_log2);
-              y[4 * i + 2] = fwd_scale(f.z, P.ep.scale_log2);
-              y[4 * i + 3] = fwd_scale(f.w, P.ep.scale_log2);
-            }
-            fwd_chunk_update(y, col_base + c * 32, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) {
+            mbar_arrive_cluster(mapa_shared(tempty_bar(acc), lead));
+          } else {
+            mbar_arrive(tempty_bar(acc));
           }
         }
-        epilogue_bar();  // Y read: free for the next block
+        mbar_arrive(xfull_bar);
+        if (warp != 2) continue;
+        if (!warp_wait(xfull_bar, k & 1u)) break;
+        float m = kMaskLogit, s = 0.f, b = 0.f;
+        if (rank > 0) {  // hfull(h, 0) has completed (waited above)
+          const float* in = hand + h * 3 * MR;
+          m = in[t];
+          s = in[MR + t];
+          b = in[2 * MR + t];
+          mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
+        }
+        const float4* row = reinterpret_cast<const float4*>(Y + lane * kDecYStride);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 f = row[c * 8 + i];
+            y[4 * i + 0] = fwd_scale(f.x, P.ep.scale_log2);
+            y[4 * i + 1] = fwd_scale(f.y, P.ep.scale_log2);
+            y[4 * i + 2] = fwd_scale(f.z, P.ep.scale_log2);
+            y[4 * i + 3] = fwd_scale(f.w, P.ep.scale_log2);
+          }
+          if (t < P.ep.T) fwd_chunk_update(y, tile0 + c * 32, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
+        }
+        mbar_arrive(xfree_bar);
+        if (rank + 1 < kDecCluster) {
+          if (!warp_wait(hempty_bar(h), hph ^ 1u)) break;
+          const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * MR), rank + 1);
+          st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
+          st_shared_cluster_u32(dst + 4u * (MR + t), __float_as_uint(s));
+          st_shared_cluster_u32(dst + 4u * (2 * MR + t), __float_as_uint(b));
+          mbar_arrive_cluster(mapa_shared(hfull_bar(h, 0), rank + 1));
+        } else if (t < P.ep.T) {
+          const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
+          P.ep.part_m[i] = m;
+          P.ep.part_s[i] = s;
+          P.ep.part_b[i] = b;
+        }
+        continue;
       }
-      // 4. hand the triple on, or store the split's triple
-      if (rank + 1 < kDecCluster) {
-        if (ep_leader) *ok3 = mbar_wait_bounded(hempty_bar(h), hph ^ 1u, abort_flag, err) ? 1 : 0;
-        epilogue_bar();
-        if (!*ok3) break;
-        const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * kDecMaxRows), rank + 1);
-        st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
-        st_shared_cluster_u32(dst + 4u * (kDecMaxRows + t), __float_as_uint(s));
-        st_shared_cluster_u32(dst + 4u * (2 * kDecMaxRows + t), __float_as_uint(b));
-        mbar_arrive_cluster(mapa_shared(hfull_bar(h), rank + 1));
-      } else if (tvalid) {
-        const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
-        P.ep.part_m[i] = m;
-        P.ep.part_s[i] = s;
-        P.ep.part_b[i] = b;
+      for (int blk = 0; blk < nblk; ++blk, ++g) {
+        const int t = blk * 32 + lane;
+        const int64_t tgt = t < P.ep.T ? P.ep.targets[t] - P.ep.v0 : -1;  // issued early
+        // 1. this block's 32 columns of the accumulator, transposed through the
+        //    warp's tile: lane l ends with batch row blk*32+l over the chunk
+        if (N == 16) {
+          uint32_t r[16];
+          tmem_ld16(tl + acc * MR, r);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) xt[lane * kDecXStride + j] = __uint_as_float(r[j]);
+        } else {
+          uint32_t r[32];
+          tmem_ld32(tl + acc * MR + blk * 32, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) xt[lane * kDecXStride + j] = __uint_as_float(r[j]);
+        }
+        if (blk == nblk - 1) {  // the accumulator's last columns are read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (kPair) {
+              mbar_arrive_cluster(mapa_shared(tempty_bar(acc), lead));
+            } else {
+              mbar_arrive(tempty_bar(acc));
+            }
+          }
+        }
+        __syncwarp();
+        float y[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) y[i] = fwd_scale(xt[i * kDecXStride + lane], P.ep.scale_log2);
+        __syncwarp();  // the tile is free for the next block
+        // 2. the rows' running triples
+        float m = kMaskLogit, s = 0.f, b = 0.f;
+        if (q == 0) {
+          if (rank > 0) {
+            if (!warp_wait_cluster(hfull_bar(h, blk), hph)) {
+              ok = false;
+              break;
+            }
+            const float* in = hand + h * 3 * MR;
+            m = in[t];
+            s = in[MR + t];
+            b = in[2 * MR + t];
+            if (blk == nblk - 1) mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
+          }
+        } else {
+          if (!warp_wait(pfull_bar(q - 1), g & 1u)) {
+            ok = false;
+            break;
+          }
+          const float* in = pass + (q - 1) * 96;
+          m = in[lane];
+          s = in[32 + lane];
+          b = in[64 + lane];
+          mbar_arrive(pempty_bar(q - 1));
+        }
+        // 3. fold this chunk
+        if (t < P.ep.T)
+          fwd_chunk_update(y, col0, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
+        // 4. pass the triples on
+        if (q < 3) {
+          if (!warp_wait(pempty_bar(q), (g & 1u) ^ 1u)) {
+            ok = false;
+            break;
+          }
+          float* out = pass + q * 96;
+          out[lane] = m;
+          out[32 + lane] = s;
+          out[64 + lane] = b;
+          mbar_arrive(pfull_bar(q));
+        } else if (rank + 1 < kDecCluster) {
+          if (blk == 0 && !warp_wait(hempty_bar(h), hph ^ 1u)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * MR), rank + 1);
+          st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
+          st_shared_cluster_u32(dst + 4u * (MR + t), __float_as_uint(s));
+          st_shared_cluster_u32(dst + 4u * (2 * MR + t), __float_as_uint(b));
+          mbar_arrive_cluster(mapa_shared(hfull_bar(h, blk), rank + 1));
+        } else if (t < P.ep.T) {
+          const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
+          P.ep.part_m[i] = m;
+          P.ep.part_s[i] = s;
+          P.ep.part_b[i] = b;
+        }
       }
     }
   }
@@ -296,19 +525,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
   if (*abort_flag) {
     // Unwind after a timed-out wait: let TMA loads and MMAs in flight finish
     // before the shared memory and TMEM they touch go away.
-    if (warp == 0 && lane == 0) {
+    if (warp == 0 && lane == 0 && is_lead) {
       const uint32_t first = issued > static_cast<uint32_t>(S) ? issued - S : 0u;
       for (uint32_t i = first; i < issued; ++i) mbar_wait_drain(full_bar(i % S), (i / S) & 1u);
     }
-    if (warp == 1 && lane == 0) {
-      umma_commit(drain_bar);
+    if (warp == 1 && lane == 0 && is_lead) {
+      if constexpr (kPair) {
+        umma_commit_pair_mask(drain_bar, pair_mask);
+      } else {
+        umma_commit(drain_bar);
+      }
       mbar_wait_drain(drain_bar, 0);
+    }
+    if constexpr (kPair) {
+      // the odd CTA's copies signal the even CTA's barriers: give them time to land
+      const uint64_t t_start = globaltimer_ns();
+      while (globaltimer_ns() - t_start < 2000000ull) __nanosleep(1000);
     }
     __syncthreads();
   }
   cluster_sync();  // no CTA exits while a neighbour may still write its shared memory
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kDecTmemCols);
+  if (warp == 1) {
+    if constexpr (kPair) {
+      tmem_dealloc_pair(tmem_base, DecForm<kPair>::kTmemCols);
+    } else {
+      tmem_dealloc(tmem_base, DecForm<kPair>::kTmemCols);
+    }
+  }
 }
 
 }  // namespace rlk

@@ -82,6 +82,40 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// sleeps in hardware (issuing nothing) until it completes or about `hint_ns`
+// have passed.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait_bounded for waiters off the critical issue path (they share the
+// SM's schedulers with the TMA producer and the MMA issuer): the same bound
+// and abort handling, sleeping between checks.
+__device__ __forceinline__ bool mbar_wait_bounded_sleep(uint32_t bar, uint32_t parity,
+                                                        volatile int* abort_flag, uint32_t* err,
+                                                        uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
 // Same, with a short limit, for the unwinding path after an abort.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -351,6 +385,16 @@ __device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
       : "memory");
 }
 
+// The same arrival for a pair anywhere in a larger cluster: `mask` has one bit
+// per CTA rank of the cluster (the pair of ranks 2 and 3 is 0b1100).
+__device__ __forceinline__ void umma_commit_pair_mask(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
 }  // namespace rlk
 
 namespace rlk {
@@ -426,6 +470,32 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t
         atomicOr(err, kDevErrTimeout);
         return false;
       }
+    }
+  }
+}
+
+// The sleeping form of mbar_wait_cluster_bounded (see mbar_wait_bounded_sleep).
+__device__ __forceinline__ bool mbar_wait_cluster_bounded_sleep(uint32_t bar, uint32_t parity,
+                                                                volatile int* abort_flag,
+                                                                uint32_t* err,
+                                                                uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(20000u)
+        : "memory");
+    if (ok) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(err, kDevErrTimeout);
+      return false;
     }
   }
 }

@@ -4,8 +4,9 @@ of a larger allocation whose 4 KB on both sides hold a byte pattern, and after
 the calls every guard byte must be unchanged.  The kernels write past ragged
 edges with TMA stores and vector stores (dX boxes at T and at chunk tails, dW
 rows at V, the dHidden accumulator, split partials), so the shapes are ragged
-on purpose: T on both sides of the 128-row short-batch switch and of the
-256-row tile, V on both sides of the 8192-row backward chunk, H at its
+on purpose: T on both sides of the switch between the two short-batch MMA
+forms (32 / 33), of the short-batch switch (224 / 225) and of the 256-row
+tile (256 / 257), V on both sides of the 8192-row backward chunk, H at its
 smallest and at the model's size.  The guarded results must also equal the
 results of the same calls on plain allocations bit for bit, and the fp64
 oracle within the parity tolerances (fail closed, zero mismatches: VIME
@@ -77,8 +78,9 @@ def _plain_step(hid, W, tg, dl, de, tau):
     return dict(logp=logp, entropy=ent, lse=lse, dH=dH, dW=dW)
 
 
-CASES = [(1, 64, 1), (127, 64, 1537), (129, 64, 8193), (255, 4096, 1537),
-         (257, 4096, 8193), (1, 4096, 151936), (129, 64, 151936)]
+CASES = [(1, 64, 1), (32, 64, 1537), (33, 64, 8193), (127, 64, 1537), (129, 64, 8193),
+         (224, 4096, 1537), (225, 64, 8193), (256, 64, 8193), (257, 4096, 8193),
+         (1, 4096, 151936), (129, 64, 151936)]
 
 
 @pytest.mark.parametrize("T,H,V", CASES)
