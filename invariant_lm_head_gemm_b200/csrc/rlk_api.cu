@@ -420,7 +420,7 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   for (int i = 0; i < kDxBuffers; ++i) {
     dx[i] = ws + L.dx[i];
     if (!map_kmajor(&P.maps.dx_k[i], dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !make_map(&P.maps.dx_st[i], dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map(&P.maps.dx_st[i], dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return RLK_ERR_CUDA;
   }
   // MN-major operands of the dHidden and dW units: 3-D maps (half the copies)

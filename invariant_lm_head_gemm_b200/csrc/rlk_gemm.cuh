@@ -191,10 +191,14 @@ struct EpiDlogits {
   }
 
   // One 128 x 256 tile, 32 columns at a time.  Each warp stages its 32 x 32
-  // bf16 block in shared memory (two 2 KB buffers, `stage`) and one lane
-  // writes it to dX[warp_row0 .. +32, col .. +32] with a TMA store (rows past
-  // T are not written).  The caller waits for the stores (bulk_wait_all)
-  // before publishing the tile.
+  // bf16 block in shared memory (two 2 KB buffers, `stage`, 1024-byte
+  // aligned) and one lane writes it to dX[warp_row0 .. +32, col .. +32] with a
+  // TMA store (rows past T are not written).  The staging layout is the
+  // store map's 64-byte swizzle: the 16-byte piece q of row r sits at piece
+  // q ^ ((r >> 1) & 3) of the row, so the warp's 16-byte stores spread over
+  // all 32 banks (a plain 64-byte row pitch puts every even lane on the same
+  // four banks).  The caller waits for the stores (bulk_wait_all) before
+  // publishing the tile.
   __device__ static void tile(const Params& p, State& st, uint32_t taddr, int nt,
                               const CUtensorMap* store_map, uint32_t stage, int lane,
                               int warp_row0) {
@@ -227,9 +231,10 @@ struct EpiDlogits {
         if (lane == 0) bulk_wait_read_le1();  // the store two chunks back has read `buf`
         __syncwarp();
         const uint32_t row_addr = buf + lane * 64u;
+        const uint32_t sw = static_cast<uint32_t>(lane >> 1) & 3u;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          st_shared_v4(row_addr + q * 16u, pack_bf16x2(dx[8 * q + 0], dx[8 * q + 1]),
+          st_shared_v4(row_addr + ((static_cast<uint32_t>(q) ^ sw) << 4), pack_bf16x2(dx[8 * q + 0], dx[8 * q + 1]),
                        pack_bf16x2(dx[8 * q + 2], dx[8 * q + 3]),
                        pack_bf16x2(dx[8 * q + 4], dx[8 * q + 5]),
                        pack_bf16x2(dx[8 * q + 6], dx[8 * q + 7]));
