@@ -441,6 +441,51 @@ def run_ours(args):
         trans["frac"].append(t_gbs / peaks()[0]["hbm_gbs"])
         del tg_graph
 
+    # ---------------------------------------------------------------- dense GEMM (LoRA-gate shapes)
+    # The batch-invariant dense GEMM on the report's LoRA-gate shapes (y[T,N] =
+    # x[T,K] . W[N,K]^T, fp32 out).  A CUDA graph of 20 calls that cycle
+    # through enough copies of x and W to exceed L2 (so W streams from HBM as
+    # it would in a model), replayed 5 times.  Bound per shape: the larger of
+    # the tensor time (2TNK at the burst peak) and the HBM time (x, W and y).
+    gemm = {"kernel": "T <= 224: decode_fwd_kernel store mode (operands swapped, 128 W rows per "
+                      "CTA); larger T: pair_kernel<kModeGemm> (256 x 256 pair tiles); fp32 out",
+            "timing": "CUDA graph of 20 calls over rotating copies (> L2), replayed 5 times",
+            "shapes": [], "us_per_call": [], "tflops": [], "gbs": [], "bound": [], "frac": []}
+    for (gN, gK, gT) in ((512, 384, 70), (2048, 1024, 257), (5120, 5120, 33)):
+        w_bytes = 2 * (gN + gT) * gK
+        ncopy = max(2, -(-256 * 2 ** 20 // w_bytes))
+        gx = [torch.randn(gT, gK, device=dev).to(torch.bfloat16) for _ in range(ncopy)]
+        gw = [(torch.randn(gN, gK, device=dev) / gK ** 0.5).to(torch.bfloat16) for _ in range(ncopy)]
+        gy = torch.empty(gT, gN, device=dev)
+        g_ws = torch.zeros(int(binding.lib().rlk_gemm_workspace_bytes()), dtype=torch.uint8,
+                           device=dev)
+        binding.rlk_gemm_bf16_f32(gx[0], gw[0], out=gy, workspace=g_ws)
+        g_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_graph, capture_error_mode="thread_local"):
+            for i in range(20):
+                binding.rlk_gemm_bf16_f32(gx[i % ncopy], gw[i % ncopy], out=gy, workspace=g_ws)
+        g_graph.replay()
+        ga0 = torch.cuda.Event(enable_timing=True)
+        ga1 = torch.cuda.Event(enable_timing=True)
+        ga0.record(stream)
+        for _ in range(5):
+            g_graph.replay()
+        ga1.record(stream)
+        torch.cuda.synchronize()
+        g_us = 1e3 * ga0.elapsed_time(ga1) / 100
+        g_flops = 2.0 * gT * gN * gK
+        g_bytes = w_bytes + 4 * gT * gN
+        t_tensor = g_flops / (peaks()[0]["bf16_tflops"] * 1e12) * 1e6
+        t_hbm = g_bytes / (peaks()[0]["hbm_gbs"] * 1e9) * 1e6
+        gemm["shapes"].append("N%d K%d T%d" % (gN, gK, gT))
+        gemm["us_per_call"].append(g_us)
+        gemm["tflops"].append(g_flops / (g_us * 1e-6) / 1e12)
+        gemm["gbs"].append(g_bytes / (g_us * 1e-6) / 1e9)
+        gemm["bound"].append("tensor" if t_tensor > t_hbm else "hbm")
+        gemm["frac"].append(max(t_tensor, t_hbm) / g_us)
+        del g_graph, gx, gw
+    gemm["device_error_flags"] = binding.rlk_read_device_error(g_ws)
+
     # ---------------------------------------------------------------- device-resident
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     for _ in range(args.warmup):
@@ -705,6 +750,7 @@ def run_ours(args):
                                                 if use_rs else 0)},
         "decode_fwd": decode,
         "transition": trans,
+        "dense_gemm": gemm,
         "tp_shard": dict(tp_line, frac=tp_line["tflops"] / pk["bf16_tflops"],
                          peak=pk["bf16_tflops"]),
         "clocks": clk.summary(),

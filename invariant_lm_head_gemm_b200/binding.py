@@ -229,17 +229,30 @@ def rlk_test_linear_logp_bwd_stall(hidden, W, targets, temperature, lse, entropy
     return dHidden, dW
 
 
-def rlk_gemm_bf16_f32(A, B, a_mn_major=False, b_mn_major=False, stream=None):
+def rlk_gemm_bf16_f32(A, B, a_mn_major=False, b_mn_major=False, stream=None, out=None,
+                      workspace=None):
     """C = A' . B'^T through the tensor-core mainloop (self-check entry).
-    A' is A ([M,K]) or A^T (A stored [K,M] when a_mn_major); B' likewise."""
+    A' is A ([M,K]) or A^T (A stored [K,M] when a_mn_major); B' likewise.
+    `out` (fp32 [M,N]) and `workspace` (zeroed uint8, rlk_gemm_workspace_bytes
+    long) may be given to reuse buffers across calls."""
     _req(A, torch.bfloat16, "A", 2)
     _req(B, torch.bfloat16, "B", 2)
     M, K = (A.shape[1], A.shape[0]) if a_mn_major else A.shape
     N, K2 = (B.shape[1], B.shape[0]) if b_mn_major else B.shape
     if K != K2:
         raise ValueError("K mismatch")
-    C = torch.empty(M, N, dtype=torch.float32, device=A.device)
-    ws = torch.zeros(int(lib().rlk_gemm_workspace_bytes()), dtype=torch.uint8, device=A.device)
+    if out is None:
+        C = torch.empty(M, N, dtype=torch.float32, device=A.device)
+    else:
+        _req(out, torch.float32, "out", 2)
+        if tuple(out.shape) != (M, N):
+            raise ValueError("out must be [M, N]")
+        C = out
+    if workspace is None:
+        ws = torch.zeros(int(lib().rlk_gemm_workspace_bytes()), dtype=torch.uint8,
+                         device=A.device)
+    else:
+        ws = workspace
     _check(lib().rlk_gemm_bf16_f32(_ptr(A), _ptr(B), M, N, K, int(a_mn_major), int(b_mn_major),
                                    _ptr(C), _ptr(ws), ws.numel(), _stream(stream)),
            "rlk_gemm_bf16_f32")

@@ -264,41 +264,23 @@ rlk_status launch_pair(const typename ModeArgs<Mode>::type& args, long long tota
 // target falls in these rows, the target's scaled logit to ytgt.
 static_assert(kDecSplit == kBN * kFwdGroup, "both forward kernels must use the same splits");
 
-std::atomic<int> g_dec_max_clusters[2][kDecMaxRows / 16][kMaxDevices];  // by form, N / 16 - 1
+std::atomic<int> g_dec_max_clusters[2][2][kDecMaxRows / 16][kMaxDevices];  // store, form, N/16-1
 
-// Forward partials for T <= kDecMaxT (decode_fwd_kernel, rlk_decode.cuh):
-// the single-CTA MMA form below N = kDecPairMinN, the CTA-pair form from there.
-rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
-                                      const int64_t* targets, int64_t T, int64_t H, int64_t Vloc,
-                                      int64_t v0, float temperature, float* part_m, float* part_s,
-                                      float* part_b, int64_t ldp, float* ytgt, uint32_t* err,
-                                      cudaStream_t st) {
-  DecArgs a;
-  a.N = T <= 16 ? 16 : static_cast<int>(ceil_div(T, 32) * 32);
+// The MMA width of the short-batch kernel for T rows: 16, or T rounded up to 32.
+int dec_width(int64_t T) { return T <= 16 ? 16 : static_cast<int>(ceil_div(T, 32) * 32); }
+
+// Launches the short-batch kernel (rlk_decode.cuh) on args whose maps, epilogue
+// fields, KB and NG are set: the single-CTA MMA form below N = kDecPairMinN, the
+// CTA-pair form from there (its hidden map's box must then hold N / 2 rows);
+// `store` selects the plain GEMM epilogue instead of the online fold.
+rlk_status launch_short(DecArgs& a, bool store, cudaStream_t st) {
   const bool pair = a.N >= kDecPairMinN;
-  // the pair form splits the N hidden rows between the two CTAs (N / 2 each)
-  if (!map_kmajor(&a.w_k, W, H, Vloc, H, kBM) ||
-      !map_kmajor(&a.hid_k, hidden, H, T, H, pair ? a.N / 2 : a.N))
-    return RLK_ERR_CUDA;
-  a.ep.targets = targets;
-  a.ep.part_m = part_m;
-  a.ep.part_s = part_s;
-  a.ep.part_b = part_b;
-  a.ep.ytgt = ytgt;
-  a.ep.T = static_cast<int>(T);
-  a.ep.V = static_cast<int>(Vloc);
-  a.ep.ldp = static_cast<int>(ldp);
-  a.ep.v0 = v0;
-  a.ep.scale_log2 = kLog2e / temperature;
-  a.err = err;
-  a.KB = static_cast<int>(H / kBK);
-  a.NG = static_cast<int>(fwd_groups(Vloc));
   constexpr uint32_t kSmemLimit = 227u * 1024u;
   a.stages = dec_stages(a.N, pair, kSmemLimit);
   if (a.stages == 0) return RLK_ERR_CUDA;
   const uint32_t smem = dec_smem_bytes(a.N, a.stages, pair);
-  void (*kern)(DecArgs) = pair ? decode_fwd_kernel<true> : decode_fwd_kernel<false>;
-
+  void (*kern)(DecArgs) = store ? (pair ? decode_fwd_kernel<true, true> : decode_fwd_kernel<false, true>)
+                                : (pair ? decode_fwd_kernel<true, false> : decode_fwd_kernel<false, false>);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
@@ -320,7 +302,7 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  std::atomic<int>& cache = g_dec_max_clusters[pair ? 1 : 0][a.N / 16 - 1][dev];
+  std::atomic<int>& cache = g_dec_max_clusters[store ? 1 : 0][pair ? 1 : 0][a.N / 16 - 1][dev];
   int mc = cache.load(std::memory_order_relaxed);
   if (mc == 0) {
     cfg.gridDim = dim3(kDecCluster);
@@ -338,6 +320,34 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
     return RLK_ERR_CUDA;
   }
   return RLK_OK;
+}
+
+// Forward partials for T <= kDecMaxT (decode_fwd_kernel, rlk_decode.cuh).
+rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
+                                      const int64_t* targets, int64_t T, int64_t H, int64_t Vloc,
+                                      int64_t v0, float temperature, float* part_m, float* part_s,
+                                      float* part_b, int64_t ldp, float* ytgt, uint32_t* err,
+                                      cudaStream_t st) {
+  DecArgs a;
+  a.N = dec_width(T);
+  const bool pair = a.N >= kDecPairMinN;
+  if (!map_kmajor(&a.w_k, W, H, Vloc, H, kBM) ||
+      !map_kmajor(&a.hid_k, hidden, H, T, H, pair ? a.N / 2 : a.N))
+    return RLK_ERR_CUDA;
+  a.ep.targets = targets;
+  a.ep.part_m = part_m;
+  a.ep.part_s = part_s;
+  a.ep.part_b = part_b;
+  a.ep.ytgt = ytgt;
+  a.ep.T = static_cast<int>(T);
+  a.ep.V = static_cast<int>(Vloc);
+  a.ep.ldp = static_cast<int>(ldp);
+  a.ep.v0 = v0;
+  a.ep.scale_log2 = kLog2e / temperature;
+  a.err = err;
+  a.KB = static_cast<int>(H / kBK);
+  a.NG = static_cast<int>(fwd_groups(Vloc));
+  return launch_short(a, false, st);
 }
 
 rlk_status enqueue_fwd_partials(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
@@ -658,6 +668,28 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(workspace);
 
+  if (!a_mn_major && !b_mn_major && M <= kDecMaxT) {
+    // Few rows: the short-batch kernel with the operands swapped (B's rows on
+    // the MMA's M side, A's M rows on its N side) and a plain store epilogue.
+    // Each C element is the same K-ordered dot product as in the pair tiles,
+    // so the results do not depend on which path a row count takes.
+    DecArgs d;
+    d.N = dec_width(M);
+    if (!map_kmajor(&d.w_k, B, K, N, K, kBM) ||
+        !map_kmajor(&d.hid_k, A, K, M, K, d.N >= kDecPairMinN ? d.N / 2 : d.N))
+      return RLK_ERR_CUDA;
+    d.ep = EpiFwd::Params{};
+    d.ep.part_m = C;
+    d.ep.T = static_cast<int>(M);
+    d.ep.V = static_cast<int>(N);
+    d.ep.ldp = static_cast<int>(N);
+    d.err = err;
+    d.KB = static_cast<int>(ceil_div(K, kBK));
+    d.NG = static_cast<int>(fwd_groups(N));
+    s = launch_short(d, true, st);
+    if (s == RLK_OK) g_calls[2].fetch_add(1);
+    return s;
+  }
   GemmArgs a;
   a.a3 = a_mn_major && map_mnmajor3(&a.a, A, M, K, M) ? 1 : 0;
   a.b3 = b_mn_major && map_mnmajor3(&a.b, B, N, K, N) ? 1 : 0;

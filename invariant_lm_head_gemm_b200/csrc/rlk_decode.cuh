@@ -91,7 +91,9 @@ struct DecForm {
 struct DecArgs {
   CUtensorMap w_k;    // W [V, H], K-major, box 64 x 128
   CUtensorMap hid_k;  // hidden [T, H], K-major, box 64 x N
-  EpiFwd::Params ep;  // outputs and layout of the pair kernel's forward
+  EpiFwd::Params ep;  // outputs and layout of the pair kernel's forward; for the
+                      // plain GEMM (kStore) part_m = C, T = rows, V = columns,
+                      // ldp = C's row stride, the rest unused
   uint32_t* err;
   int N;              // MMA N: 16 for T <= 16, else T rounded up to 32
                       // (the hidden box holds N rows, or N / 2 in the pair form)
@@ -117,7 +119,7 @@ __host__ __device__ constexpr int dec_stages(int N, bool pair, uint32_t limit) {
   return S >= 2 ? S : 0;
 }
 
-template <bool kPair>
+template <bool kPair, bool kStore = false>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid_constant__ DecArgs P) {
   constexpr int MR = DecForm<kPair>::kMaxRows;  // batch rows a hand buffer holds
   extern __shared__ uint8_t smem_raw[];
@@ -339,113 +341,91 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
       return ok != 0;
     };
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    uint32_t g = 0;  // blocks this warp has passed on (phase of its links)
     bool ok = true;
-    for (uint32_t k = 0; ok; ++k) {
-      const long long u = unit_of(k);
-      if (u < 0) break;
-      const int acc = k & 1, h = k & 1;
-      const uint32_t hph = (k >> 1) & 1u;
-      if (!warp_wait(tfull_bar(acc), hph)) break;
-      tc_fence_after();
-      const int tile0 = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
-      const int col0 = tile0 + q * 32;
-      if (nblk == 1) {
-        // One 32-row block (N <= 32): every warp transposes its chunk, then
-        // warp 2 folds all four in order.  Passing the rows from warp to warp
-        // would overlap nothing here and only lengthen the chain of CTAs by
-        // three hand-offs; and warp 2 is the epilogue warp that shares its
-        // scheduler with neither the producer (warp 0) nor the MMA issuer
-        // (warp 1), whose issue latency sets the W stream.
-        // The accumulator is read once the running triples have arrived from
-        // CTA rank-1: releasing it sooner lets the four CTAs of a split drift
-        // apart in their W streams, which measured ~2% slower.  The tile is
-        // row-major per batch row (Y[row][W row of the tile]), in the memory of
-        // the four transposition tiles.
-        const int t = lane;
-        const int64_t tgt = t < P.ep.T ? P.ep.targets[t] - P.ep.v0 : -1;
-        float* Y = XT;
-        if (warp != 2 && k > 0 && !warp_wait(xfree_bar, (k - 1) & 1u)) break;
-        if (rank > 0 && !warp_wait_cluster(hfull_bar(h, 0), hph)) break;
-        const int v_loc = q * 32 + lane;
-        if (N == 16) {
-          uint32_t r[16];
-          tmem_ld16(tl + acc * MR, r);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
-        } else {
+    if constexpr (kStore) {
+      // The plain GEMM (C[T, V] = hidden . W^T, fp32): lane l of warp q holds
+      // output column n = tile row 32q + l for the accumulator's batch rows;
+      // each row t is stored as one coalesced 128-byte run of the warp.
+      float* C = P.ep.part_m;
+      for (uint32_t k = 0; ok; ++k) {
+        const long long u = unit_of(k);
+        if (u < 0) break;
+        const int acc = k & 1;
+        if (!warp_wait(tfull_bar(acc), (k >> 1) & 1u)) break;
+        tc_fence_after();
+        const int n = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM + q * 32 + lane;
+        for (int blk = 0; blk < nblk; ++blk) {
           uint32_t r[32];
-          tmem_ld32(tl + acc * MR, r);
+          const int cols = N == 16 ? 16 : 32;
+          if (N == 16) {
+            uint32_t r16[16];
+            tmem_ld16(tl + acc * MR, r16);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (kPair) {
-            mbar_arrive_cluster(mapa_shared(tempty_bar(acc), lead));
+            for (int j = 0; j < 16; ++j) r[j] = r16[j];
           } else {
-            mbar_arrive(tempty_bar(acc));
+            tmem_ld32(tl + acc * MR + blk * 32, r);
           }
-        }
-        mbar_arrive(xfull_bar);
-        if (warp != 2) continue;
-        if (!warp_wait(xfull_bar, k & 1u)) break;
-        float m = kMaskLogit, s = 0.f, b = 0.f;
-        if (rank > 0) {  // hfull(h, 0) has completed (waited above)
-          const float* in = hand + h * 3 * MR;
-          m = in[t];
-          s = in[MR + t];
-          b = in[2 * MR + t];
-          mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
-        }
-        const float4* row = reinterpret_cast<const float4*>(Y + lane * kDecYStride);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float y[32];
+          if (blk == nblk - 1) {  // the accumulator's last columns are read
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (kPair) {
+                mbar_arrive_cluster(mapa_shared(tempty_bar(acc), lead));
+              } else {
+                mbar_arrive(tempty_bar(acc));
+              }
+            }
+          }
+          if (n < P.ep.V) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 f = row[c * 8 + i];
-            y[4 * i + 0] = fwd_scale(f.x, P.ep.scale_log2);
-            y[4 * i + 1] = fwd_scale(f.y, P.ep.scale_log2);
-            y[4 * i + 2] = fwd_scale(f.z, P.ep.scale_log2);
-            y[4 * i + 3] = fwd_scale(f.w, P.ep.scale_log2);
+            for (int j = 0; j < 32; ++j) {
+              const int t = blk * 32 + j;
+              if (j < cols && t < P.ep.T)
+                C[static_cast<size_t>(t) * P.ep.ldp + n] = __uint_as_float(r[j]);
+            }
           }
-          if (t < P.ep.T) fwd_chunk_update(y, tile0 + c * 32, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
         }
-        mbar_arrive(xfree_bar);
-        if (rank + 1 < kDecCluster) {
-          if (!warp_wait(hempty_bar(h), hph ^ 1u)) break;
-          const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * MR), rank + 1);
-          st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
-          st_shared_cluster_u32(dst + 4u * (MR + t), __float_as_uint(s));
-          st_shared_cluster_u32(dst + 4u * (2 * MR + t), __float_as_uint(b));
-          mbar_arrive_cluster(mapa_shared(hfull_bar(h, 0), rank + 1));
-        } else if (t < P.ep.T) {
-          const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
-          P.ep.part_m[i] = m;
-          P.ep.part_s[i] = s;
-          P.ep.part_b[i] = b;
-        }
-        continue;
       }
-      for (int blk = 0; blk < nblk; ++blk, ++g) {
-        const int t = blk * 32 + lane;
-        const int64_t tgt = t < P.ep.T ? P.ep.targets[t] - P.ep.v0 : -1;  // issued early
-        // 1. this block's 32 columns of the accumulator, transposed through the
-        //    warp's tile: lane l ends with batch row blk*32+l over the chunk
-        if (N == 16) {
-          uint32_t r[16];
-          tmem_ld16(tl + acc * MR, r);
+    } else {
+      uint32_t g = 0;  // blocks this warp has passed on (phase of its links)
+      for (uint32_t k = 0; ok; ++k) {
+        const long long u = unit_of(k);
+        if (u < 0) break;
+        const int acc = k & 1, h = k & 1;
+        const uint32_t hph = (k >> 1) & 1u;
+        if (!warp_wait(tfull_bar(acc), hph)) break;
+        tc_fence_after();
+        const int tile0 = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
+        const int col0 = tile0 + q * 32;
+        if (nblk == 1) {
+          // One 32-row block (N <= 32): every warp transposes its chunk, then
+          // warp 2 folds all four in order.  Passing the rows from warp to warp
+          // would overlap nothing here and only lengthen the chain of CTAs by
+          // three hand-offs; and warp 2 is the epilogue warp that shares its
+          // scheduler with neither the producer (warp 0) nor the MMA issuer
+          // (warp 1), whose issue latency sets the W stream.
+          // The accumulator is read once the running triples have arrived from
+          // CTA rank-1: releasing it sooner lets the four CTAs of a split drift
+          // apart in their W streams, which measured ~2% slower.  The tile is
+          // row-major per batch row (Y[row][W row of the tile]), in the memory of
+          // the four transposition tiles.
+          const int t = lane;
+          const int64_t tgt = t < P.ep.T ? P.ep.targets[t] - P.ep.v0 : -1;
+          float* Y = XT;
+          if (warp != 2 && k > 0 && !warp_wait(xfree_bar, (k - 1) & 1u)) break;
+          if (rank > 0 && !warp_wait_cluster(hfull_bar(h, 0), hph)) break;
+          const int v_loc = q * 32 + lane;
+          if (N == 16) {
+            uint32_t r[16];
+            tmem_ld16(tl + acc * MR, r);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) xt[lane * kDecXStride + j] = __uint_as_float(r[j]);
-        } else {
-          uint32_t r[32];
-          tmem_ld32(tl + acc * MR + blk * 32, r);
+            for (int j = 0; j < 16; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
+          } else {
+            uint32_t r[32];
+            tmem_ld32(tl + acc * MR, r);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) xt[lane * kDecXStride + j] = __uint_as_float(r[j]);
-        }
-        if (blk == nblk - 1) {  // the accumulator's last columns are read
+            for (int j = 0; j < 32; ++j) Y[j * kDecYStride + v_loc] = __uint_as_float(r[j]);
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
@@ -455,66 +435,134 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
               mbar_arrive(tempty_bar(acc));
             }
           }
-        }
-        __syncwarp();
-        float y[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) y[i] = fwd_scale(xt[i * kDecXStride + lane], P.ep.scale_log2);
-        __syncwarp();  // the tile is free for the next block
-        // 2. the rows' running triples
-        float m = kMaskLogit, s = 0.f, b = 0.f;
-        if (q == 0) {
-          if (rank > 0) {
-            if (!warp_wait_cluster(hfull_bar(h, blk), hph)) {
-              ok = false;
-              break;
-            }
+          mbar_arrive(xfull_bar);
+          if (warp != 2) continue;
+          if (!warp_wait(xfull_bar, k & 1u)) break;
+          float m = kMaskLogit, s = 0.f, b = 0.f;
+          if (rank > 0) {  // hfull(h, 0) has completed (waited above)
             const float* in = hand + h * 3 * MR;
             m = in[t];
             s = in[MR + t];
             b = in[2 * MR + t];
-            if (blk == nblk - 1) mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
+            mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
           }
-        } else {
-          if (!warp_wait(pfull_bar(q - 1), g & 1u)) {
-            ok = false;
-            break;
+          const float4* row = reinterpret_cast<const float4*>(Y + lane * kDecYStride);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float y[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 f = row[c * 8 + i];
+              y[4 * i + 0] = fwd_scale(f.x, P.ep.scale_log2);
+              y[4 * i + 1] = fwd_scale(f.y, P.ep.scale_log2);
+              y[4 * i + 2] = fwd_scale(f.z, P.ep.scale_log2);
+              y[4 * i + 3] = fwd_scale(f.w, P.ep.scale_log2);
+            }
+            if (t < P.ep.T) fwd_chunk_update(y, tile0 + c * 32, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
           }
-          const float* in = pass + (q - 1) * 96;
-          m = in[lane];
-          s = in[32 + lane];
-          b = in[64 + lane];
-          mbar_arrive(pempty_bar(q - 1));
+          mbar_arrive(xfree_bar);
+          if (rank + 1 < kDecCluster) {
+            if (!warp_wait(hempty_bar(h), hph ^ 1u)) break;
+            const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * MR), rank + 1);
+            st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
+            st_shared_cluster_u32(dst + 4u * (MR + t), __float_as_uint(s));
+            st_shared_cluster_u32(dst + 4u * (2 * MR + t), __float_as_uint(b));
+            mbar_arrive_cluster(mapa_shared(hfull_bar(h, 0), rank + 1));
+          } else if (t < P.ep.T) {
+            const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
+            P.ep.part_m[i] = m;
+            P.ep.part_s[i] = s;
+            P.ep.part_b[i] = b;
+          }
+          continue;
         }
-        // 3. fold this chunk
-        if (t < P.ep.T)
-          fwd_chunk_update(y, col0, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
-        // 4. pass the triples on
-        if (q < 3) {
-          if (!warp_wait(pempty_bar(q), (g & 1u) ^ 1u)) {
-            ok = false;
-            break;
+        for (int blk = 0; blk < nblk; ++blk, ++g) {
+          const int t = blk * 32 + lane;
+          const int64_t tgt = t < P.ep.T ? P.ep.targets[t] - P.ep.v0 : -1;  // issued early
+          // 1. this block's 32 columns of the accumulator, transposed through the
+          //    warp's tile: lane l ends with batch row blk*32+l over the chunk
+          if (N == 16) {
+            uint32_t r[16];
+            tmem_ld16(tl + acc * MR, r);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xt[lane * kDecXStride + j] = __uint_as_float(r[j]);
+          } else {
+            uint32_t r[32];
+            tmem_ld32(tl + acc * MR + blk * 32, r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xt[lane * kDecXStride + j] = __uint_as_float(r[j]);
           }
-          float* out = pass + q * 96;
-          out[lane] = m;
-          out[32 + lane] = s;
-          out[64 + lane] = b;
-          mbar_arrive(pfull_bar(q));
-        } else if (rank + 1 < kDecCluster) {
-          if (blk == 0 && !warp_wait(hempty_bar(h), hph ^ 1u)) {
-            ok = false;
-            break;
+          if (blk == nblk - 1) {  // the accumulator's last columns are read
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (kPair) {
+                mbar_arrive_cluster(mapa_shared(tempty_bar(acc), lead));
+              } else {
+                mbar_arrive(tempty_bar(acc));
+              }
+            }
           }
-          const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * MR), rank + 1);
-          st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
-          st_shared_cluster_u32(dst + 4u * (MR + t), __float_as_uint(s));
-          st_shared_cluster_u32(dst + 4u * (2 * MR + t), __float_as_uint(b));
-          mbar_arrive_cluster(mapa_shared(hfull_bar(h, blk), rank + 1));
-        } else if (t < P.ep.T) {
-          const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
-          P.ep.part_m[i] = m;
-          P.ep.part_s[i] = s;
-          P.ep.part_b[i] = b;
+          __syncwarp();
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = fwd_scale(xt[i * kDecXStride + lane], P.ep.scale_log2);
+          __syncwarp();  // the tile is free for the next block
+          // 2. the rows' running triples
+          float m = kMaskLogit, s = 0.f, b = 0.f;
+          if (q == 0) {
+            if (rank > 0) {
+              if (!warp_wait_cluster(hfull_bar(h, blk), hph)) {
+                ok = false;
+                break;
+              }
+              const float* in = hand + h * 3 * MR;
+              m = in[t];
+              s = in[MR + t];
+              b = in[2 * MR + t];
+              if (blk == nblk - 1) mbar_arrive_cluster(mapa_shared(hempty_bar(h), rank - 1));
+            }
+          } else {
+            if (!warp_wait(pfull_bar(q - 1), g & 1u)) {
+              ok = false;
+              break;
+            }
+            const float* in = pass + (q - 1) * 96;
+            m = in[lane];
+            s = in[32 + lane];
+            b = in[64 + lane];
+            mbar_arrive(pempty_bar(q - 1));
+          }
+          // 3. fold this chunk
+          if (t < P.ep.T)
+            fwd_chunk_update(y, col0, P.ep.V, tgt, P.ep.ytgt + t, m, s, b);
+          // 4. pass the triples on
+          if (q < 3) {
+            if (!warp_wait(pempty_bar(q), (g & 1u) ^ 1u)) {
+              ok = false;
+              break;
+            }
+            float* out = pass + q * 96;
+            out[lane] = m;
+            out[32 + lane] = s;
+            out[64 + lane] = b;
+            mbar_arrive(pfull_bar(q));
+          } else if (rank + 1 < kDecCluster) {
+            if (blk == 0 && !warp_wait(hempty_bar(h), hph ^ 1u)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = mapa_shared(smem_u32(hand + h * 3 * MR), rank + 1);
+            st_shared_cluster_u32(dst + 4u * t, __float_as_uint(m));
+            st_shared_cluster_u32(dst + 4u * (MR + t), __float_as_uint(s));
+            st_shared_cluster_u32(dst + 4u * (2 * MR + t), __float_as_uint(b));
+            mbar_arrive_cluster(mapa_shared(hfull_bar(h, blk), rank + 1));
+          } else if (t < P.ep.T) {
+            const size_t i = static_cast<size_t>(t) * P.ep.ldp + static_cast<size_t>(u);
+            P.ep.part_m[i] = m;
+            P.ep.part_s[i] = s;
+            P.ep.part_b[i] = b;
+          }
         }
       }
     }

@@ -48,3 +48,23 @@ def test_gemm_repeatable():
     for _ in range(3):
         C1, _ = binding.rlk_gemm_bf16_f32(A, B)
         assert torch.equal(C0, C1)
+
+
+@pytest.mark.parametrize("N,K", [(264, 136), (520, 4096), (8, 8), (5120, 640)])
+def test_short_row_counts_equal_rows_of_a_long_gemm(N, K):
+    """GEMMs of at most 224 rows (row-major operands) run the short-batch kernel
+    with the operands swapped and a plain store epilogue; every row must equal
+    that row of a 300-row GEMM, which runs the pair tiles, bit for bit."""
+    g = torch.Generator().manual_seed(N + K)
+    A = torch.randn(300, K, generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16).cuda()
+    full, ws = binding.rlk_gemm_bf16_f32(A, B)
+    torch.cuda.synchronize()
+    assert binding.rlk_read_device_error(ws) == 0
+    gen = torch.Generator().manual_seed(K)
+    for T in (1, 16, 17, 32, 33, 64, 100, 224):
+        rows = torch.randperm(300, generator=gen)[:T].cuda()
+        sub, ws = binding.rlk_gemm_bf16_f32(A[rows].contiguous(), B)
+        torch.cuda.synchronize()
+        assert binding.rlk_read_device_error(ws) == 0
+        assert torch.equal(sub.view(torch.int32), full[rows].view(torch.int32)), T
