@@ -281,7 +281,10 @@ rlk_status rlk_transition_logp(const float* x, const float* v, const float* prev
  * b200 report).  a_mn_major == 0: A is stored [M,K] (K contiguous); != 0:
  * stored [K,M].  b_mn_major == 0: B is stored [N,K]; != 0: stored [K,N].
  * M, N, K >= 1; K and N multiples of 8, and M too when a_mn_major.  Needs a
- * workspace of rlk_gemm_workspace_bytes() bytes for its error word. */
+ * workspace of rlk_gemm_workspace_bytes() bytes for its error word.  With
+ * row-major A and B and M <= 224 it runs the short-batch forward kernel's
+ * mainloop (operands swapped) with a plain store; every element is the same
+ * K-ordered dot product either way, so C's bits do not depend on M. */
 size_t rlk_gemm_workspace_bytes(void);
 rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, int64_t N,
                              int64_t K, int a_mn_major, int b_mn_major, float* C,
