@@ -19,10 +19,13 @@
 //    over CTAs (2i, 2i+1) of the cluster; each CTA still holds its own 128 W
 //    rows but only half of the N hidden rows (B is split along N across the
 //    pair), and each CTA's TMEM receives its 128 W rows x all N columns, so
-//    the epilogue is the same.  Halving the hidden bytes per CTA leaves room
-//    for more stages of W in flight (N = 128: four instead of three) and lets
-//    N reach 256 (three stages), where the single form would hold 64 KB of
-//    hidden per stage.
+//    the epilogue is the same.  Halving the hidden bytes per CTA lets N reach
+//    224 (three stages) where the single form would hold 56 KB of hidden per
+//    stage, and gives N = 128 four stages instead of three.
+//
+// A second epilogue (kStore) turns the kernel into the short-row path of the
+// plain dense GEMM: no fold and no chain, each accumulator column is stored
+// as C[t][n] (coalesced across the lanes of a warp).
 //
 // Numerics are those of the pair kernel, bit for bit:
 //  * each logit is the same bf16 dot product over H in the same 64-wide K
@@ -40,7 +43,7 @@
 //
 // Warp roles per CTA (192 threads): warp 0 producer (TMA), warp 1 MMA issuer
 // (in the pair form only the even CTA of each pair issues), warps 2-5
-// epilogue.  Two TMEM accumulators of up to 128 (single) or 256 (pair)
+// epilogue (the fold below, or the store of kStore).  Two TMEM accumulators of up to 128 (single) or 256 (pair)
 // columns.  The epilogue is a pipeline over 32-row batch blocks: the warp
 // that reads TMEM lane quarter q holds chunk q of the tile, transposes its
 // 32 x 32 block through its own shared-memory tile so that each lane holds one

@@ -225,3 +225,26 @@ def test_transition_step_writes_nothing_outside_its_buffers():
     assert all(g.intact() for g in (g_ws, g_mean, g_prev, g_lp))
     for p, q in zip(out, ref):
         assert torch.equal(_bits(p), _bits(q))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 8), (33, 520, 136), (224, 264, 4096), (225, 264, 136),
+                                   (70, 512, 384)])
+def test_dense_gemm_writes_nothing_outside_its_output(M, N, K):
+    """The dense GEMM's two paths (the short-batch kernel's store mode up to 224
+    rows, the pair tiles above) with ragged M, N and K: C and the workspace
+    guarded, C equal to the same call on plain allocations bit for bit and to
+    an fp64 matmul within 1e-5."""
+    g = torch.Generator().manual_seed(M + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16).cuda()
+    g_c = Guarded(4 * M * N)
+    g_ws = Guarded(int(binding.lib().rlk_gemm_workspace_bytes()), fill=0)
+    C = g_c.view(torch.float32, M, N)
+    binding.rlk_gemm_bf16_f32(A, B, out=C, workspace=g_ws.view(torch.uint8, g_ws.n))
+    ref, ws = binding.rlk_gemm_bf16_f32(A, B)
+    torch.cuda.synchronize()
+    assert binding.rlk_read_device_error(ws) == 0
+    assert g_c.intact() and g_ws.intact()
+    assert torch.equal(_bits(C), _bits(ref))
+    exact = A.double() @ B.double().t()
+    assert float((C.double() - exact).norm() / exact.norm()) < 1e-5
