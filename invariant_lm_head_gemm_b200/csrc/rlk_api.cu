@@ -178,7 +178,25 @@ bool map_mnmajor3(CUtensorMap* m, const void* base, int64_t MN, int64_t K, int64
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// K-major operand [rows, K] (K contiguous): one 64 x box_rows box per stage.
+// K-major operand [rows, K] (K contiguous, pitch elements per row) mapped 3-D
+// as (64 K, rows, K / 64) with box 64 x 128 x 2: one copy lands two K blocks of
+// 128 rows as two 16 KB swizzled blocks back to back, the same bytes and layout
+// as two 2-D boxes.  Needs K % 64 == 0 (a 2-D box fills zeros past K, this map
+// would read on into the next row); false if the driver declines the map.
+bool map_kmajor3(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t pitch) {
+  if (K % 64 != 0) return false;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(pitch) * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kBM), 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K-major operand [rows, K] (K contiguous): one 64 x box_rows box per K block.
 bool map_kmajor(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t pitch,
                 uint32_t box_rows) {
   return make_map(m, base, K, rows, pitch, 64, box_rows);
@@ -358,7 +376,10 @@ rlk_status enqueue_fwd_partials(const rlk_bf16* hidden, const rlk_bf16* W, const
     return enqueue_fwd_partials_short(hidden, W, targets, T, H, Vloc, v0, temperature, part_m,
                                       part_s, part_b, ldp, ytgt, err, st);
   FwdArgs a;
-  if (!map_kmajor(&a.hid_k, hidden, H, T, H, kBM) || !map_kmajor(&a.w_k, W, H, Vloc, H, kBM))
+  // 3-D maps (one copy per operand and stage) when the driver takes them
+  a.k3 = map_kmajor3(&a.hid_k, hidden, H, T, H) && map_kmajor3(&a.w_k, W, H, Vloc, H) ? 1 : 0;
+  if (!a.k3 &&
+      (!map_kmajor(&a.hid_k, hidden, H, T, H, kBM) || !map_kmajor(&a.w_k, W, H, Vloc, H, kBM)))
     return RLK_ERR_CUDA;
   a.ep.targets = targets;
   a.ep.part_m = part_m;
@@ -423,16 +444,19 @@ rlk_status enqueue_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t*
   BwdParams P;
   P.plan = make_bwd_plan(T, H, Vloc, vchunk(Vfull));
   const BwdPlan& pl = P.plan;
-  if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
-      !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM))
-    return RLK_ERR_CUDA;
   void* dx[kDxBuffers];
   for (int i = 0; i < kDxBuffers; ++i) {
     dx[i] = ws + L.dx[i];
-    if (!map_kmajor(&P.maps.dx_k[i], dx[i], pl.ldx, T, pl.ldx, kBM) ||
-        !make_map(&P.maps.dx_st[i], dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map(&P.maps.dx_st[i], dx[i], pl.ldx, T, pl.ldx, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return RLK_ERR_CUDA;
   }
+  // K-major operands of the recompute and dHidden units: one 2-D box per K
+  // block (the forward's one-copy 3-D stages made this kernel 1.7% slower)
+  if (!map_kmajor(&P.maps.hid_k, hidden, H, T, H, kBM) ||
+      !map_kmajor(&P.maps.w_k, W, H, Vloc, H, kBM))
+    return RLK_ERR_CUDA;
+  for (int i = 0; i < kDxBuffers; ++i)
+    if (!map_kmajor(&P.maps.dx_k[i], dx[i], pl.ldx, T, pl.ldx, kBM)) return RLK_ERR_CUDA;
   // MN-major operands of the dHidden and dW units: 3-D maps (half the copies)
   // when the driver takes them, else 2-D maps; same shared-memory bytes.
   bool mn3 = map_mnmajor3(&P.maps.w_mn, W, H, Vloc, H) &&
@@ -693,9 +717,12 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
   GemmArgs a;
   a.a3 = a_mn_major && map_mnmajor3(&a.a, A, M, K, M) ? 1 : 0;
   a.b3 = b_mn_major && map_mnmajor3(&a.b, B, N, K, N) ? 1 : 0;
-  bool ok = a.a3 || (a_mn_major ? map_mnmajor(&a.a, A, M, K, M) : map_kmajor(&a.a, A, K, M, K, kBM));
-  ok = ok && (a.b3 || (b_mn_major ? map_mnmajor(&a.b, B, N, K, N)
-                                  : map_kmajor(&a.b, B, K, N, K, kBM)));
+  a.ak3 = !a_mn_major && map_kmajor3(&a.a, A, K, M, K) ? 1 : 0;
+  a.bk3 = !b_mn_major && map_kmajor3(&a.b, B, K, N, K) ? 1 : 0;
+  bool ok = a.a3 || a.ak3 ||
+            (a_mn_major ? map_mnmajor(&a.a, A, M, K, M) : map_kmajor(&a.a, A, K, M, K, kBM));
+  ok = ok && (a.b3 || a.bk3 ||
+              (b_mn_major ? map_mnmajor(&a.b, B, N, K, N) : map_kmajor(&a.b, B, K, N, K, kBM)));
   if (!ok) return RLK_ERR_CUDA;
   a.ep.out = C;
   a.ep.rows = static_cast<int>(M);

@@ -37,7 +37,7 @@ constexpr int kDxBuffers = 3;
 
 struct BwdMaps {
   CUtensorMap hid_k;              // hidden [T,H], K-major, box 64 x 128
-  CUtensorMap w_k;                // W [V,H], K-major, box 64 x 256
+  CUtensorMap w_k;                // W [V,H], K-major, box 64 x 128
   CUtensorMap w_mn;               // W read as MN-major (N = h, K = v), box 64 x 64 (x 2 when 3-D)
   CUtensorMap hid_mn;             // hidden read as MN-major (N = h, K = t), box 64 x 64 (x 2)
   CUtensorMap dx_k[kDxBuffers];   // dX buffer [T, ldx], K-major, box 64 x 128

@@ -55,8 +55,8 @@ struct PipeCfg {
 enum : int { kJobFwd = 3, kJobGemm = 4 };  // backward jobs use kUnitR / kUnitH / kUnitD
 
 struct FwdArgs {
-  CUtensorMap hid_k;  // hidden [T,H], box 64 x 128
-  CUtensorMap w_k;    // W [V,H], box 64 x 128
+  CUtensorMap hid_k;  // hidden [T,H], box 64 x 128 (64 x 128 x 2 when k3)
+  CUtensorMap w_k;    // W [V,H], box 64 x 128 (64 x 128 x 2 when k3)
   EpiFwd::Params ep;
   uint32_t* err;
   int MT;             // 256-row M tiles
@@ -64,6 +64,7 @@ struct FwdArgs {
   int group;          // vocab tiles per unit
   int NG;             // vocab splits = ceil(NT / group)
   int KB;             // K blocks (H / 64)
+  int k3;             // both maps 3-D: one copy per operand and stage
   long long total;    // MT * NG
 };
 
@@ -75,6 +76,7 @@ struct GemmArgs {
   int M, N, MT, NT, KB;
   int a_mn, b_mn;
   int a3, b3;
+  int ak3, bk3;       // K-major operand mapped 3-D (one copy per stage)
   long long total;
 };
 
@@ -103,6 +105,8 @@ struct Job {
   int kbs;          // K blocks per tile
   bool a_mn, b_mn;  // operand majorness
   bool a3, b3;      // MN-major operand mapped 3-D: one box per 128 MN columns (else two 2-D boxes)
+  bool ak3, bk3;    // K-major operand mapped 3-D (64 K, rows, K / 64) with box 64 x 128 x 2:
+                    // one copy lands a stage's two K blocks (else one 2-D box per K block)
   const CUtensorMap* mA;
   const CUtensorMap* mB;
   int a_row0;       // M coordinate of the tile's first row in A's tensor map
@@ -123,6 +127,7 @@ __device__ __forceinline__ Job make_job(const FwdArgs& P, long long u) {
   j.kbs = P.KB;
   j.a_mn = j.b_mn = false;
   j.a3 = j.b3 = false;
+  j.ak3 = j.bk3 = P.k3 != 0;
   j.mA = &P.hid_k;
   j.mB = &P.w_k;
   j.a_row0 = j.mt * kPairM;
@@ -145,6 +150,8 @@ __device__ __forceinline__ Job make_job(const GemmArgs& P, long long u) {
   j.b_mn = P.b_mn != 0;
   j.a3 = P.a3 != 0;
   j.b3 = P.b3 != 0;
+  j.ak3 = P.ak3 != 0;
+  j.bk3 = P.bk3 != 0;
   j.mA = &P.a;
   j.mB = &P.b;
   j.a_row0 = j.mt * kPairM;
@@ -166,6 +173,7 @@ __device__ __forceinline__ Job make_job(const BwdParams& P, long long u) {
   j.ntiles = 1;
   j.bk0 = 0;
   j.a3 = j.b3 = false;
+  j.ak3 = j.bk3 = false;
   const int buf = un.c % kDxBuffers;
   if (un.type == kUnitR) {
     j.kbs = pl.KB_R;
@@ -218,26 +226,29 @@ __device__ __forceinline__ int stage_kblocks(int kbs, int st) {
   return min(kSubK, kbs - st * kSubK);
 }
 
-// Bytes CTA `rank` loads per K block (not per stage) of tile `t` of the job.
-__device__ __forceinline__ uint32_t job_bytes(const Job& j, int t, uint32_t rank) {
+// Bytes CTA `rank` loads in a stage of `nsub` K blocks of tile `t` of the job.
+// A 3-D K-major box always lands both K blocks of a stage (a second block
+// past K is filled, and a box counts in full), so it counts twice whatever
+// nsub is; the other boxes count once per K block.
+__device__ __forceinline__ uint32_t stage_bytes(const Job& j, int t, uint32_t rank, int nsub) {
   uint32_t bytes = 0;
   const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
   if (!j.a_mn) {
-    if (a0 < j.a_ext) bytes += kSubA;
+    if (a0 < j.a_ext) bytes += j.ak3 ? kSubK * kSubA : nsub * kSubA;
   } else if (j.a3) {
-    if (a0 < j.a_ext) bytes += 2 * kBox;  // the box counts in full, past-the-end half filled
+    if (a0 < j.a_ext) bytes += nsub * 2 * kBox;  // the box counts in full, past-the-end half filled
   } else {
-    if (a0 < j.a_ext) bytes += kBox;
-    if (a0 + 64 < j.a_ext) bytes += kBox;
+    if (a0 < j.a_ext) bytes += nsub * kBox;
+    if (a0 + 64 < j.a_ext) bytes += nsub * kBox;
   }
   const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
   if (!j.b_mn) {
-    if (b0 < j.b_ext) bytes += kSubB;
+    if (b0 < j.b_ext) bytes += j.bk3 ? kSubK * kSubB : nsub * kSubB;
   } else if (j.b3) {
-    if (b0 < j.b_ext) bytes += 2 * kBox;
+    if (b0 < j.b_ext) bytes += nsub * 2 * kBox;
   } else {
-    if (b0 < j.b_ext) bytes += kBox;
-    if (b0 + 64 < j.b_ext) bytes += kBox;
+    if (b0 < j.b_ext) bytes += nsub * kBox;
+    if (b0 + 64 < j.b_ext) bytes += nsub * kBox;
   }
   return bytes;
 }
@@ -388,40 +399,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; ok && t < j.ntiles; ++t) {
           const int a0 = j.a_row0 + kBM * static_cast<int>(rank);
           const int b0 = j.b_col0 + t * kBN + kBM * static_cast<int>(rank);
-          const uint32_t bytes_all = leader ? job_bytes(j, t, 0) + job_bytes(j, t, 1) : 0u;
           const int nst = (j.kbs + kSubK - 1) / kSubK;
+          // the leader's expected bytes of a full stage and of the last one,
+          // worked out once per tile (they sit on the path from a free stage
+          // to its copies)
+          const uint32_t bytes_full =
+              leader ? stage_bytes(j, t, 0, kSubK) + stage_bytes(j, t, 1, kSubK) : 0u;
+          const int nsub_last = stage_kblocks(j.kbs, nst - 1);
+          const uint32_t bytes_last =
+              leader ? stage_bytes(j, t, 0, nsub_last) + stage_bytes(j, t, 1, nsub_last) : 0u;
+          // A stage's copies are issued the moment its slot is free: everything
+          // they need is worked out before the wait, and the leader arms the
+          // full barrier after its own copies (its transaction count may run
+          // below zero meanwhile, as it does whenever the peer's copies land
+          // first).  In the load-bound backward this path sets when each
+          // load starts.
+          int s = static_cast<int>(issued % kPStages);
+          uint32_t ph = (issued / kPStages) & 1u;
           for (int st = 0; st < nst; ++st) {
-            const int s = issued % kPStages;
-            const uint32_t ph = (issued / kPStages) & 1u;
+            const int nsub = stage_kblocks(j.kbs, st);
+            const uint32_t fb = mapa_shared(full_bar(s), 0);
+            const uint32_t dA = sA + s * kPAStage, dB = sB + s * kPBStage;
+            const int k0 = st * kSubK * kBK, k1 = k0 + kBK;
+            const uint32_t bytes = st + 1 < nst ? bytes_full : bytes_last;
             if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err, lim)) {
               ok = false;
               break;
             }
-            const int nsub = stage_kblocks(j.kbs, st);
-            const uint32_t fb = mapa_shared(full_bar(s), 0);
-            if (leader) mbar_arrive_expect_tx(full_bar(s), static_cast<uint32_t>(nsub) * bytes_all);
+            // 3-D K-major operands: one copy of the stage's two K blocks
+            if (!j.a_mn && j.ak3 && a0 < j.a_ext)
+              tma_load_3d_pair(dA, j.mA, fb, 0, a0, st * kSubK);
+            if (!j.b_mn && j.bk3 && b0 < j.b_ext)
+              tma_load_3d_pair(dB, j.mB, fb, 0, b0, st * kSubK);
             for (int sub = 0; sub < nsub; ++sub) {
-              const uint32_t dA = sA + s * kPAStage + sub * kSubA;
-              const uint32_t dB = sB + s * kPBStage + sub * kSubB;
-              const int k = (st * kSubK + sub) * kBK;
+              const uint32_t dAs = dA + sub * kSubA, dBs = dB + sub * kSubB;
+              const int k = sub == 0 ? k0 : k1;
               if (!j.a_mn) {
-                if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, k, a0);
+                if (!j.ak3 && a0 < j.a_ext) tma_load_2d_pair(dAs, j.mA, fb, k, a0);
               } else if (j.a3) {
-                if (a0 < j.a_ext) tma_load_3d_pair(dA, j.mA, fb, 0, k, a0 >> 6);
+                if (a0 < j.a_ext) tma_load_3d_pair(dAs, j.mA, fb, 0, k, a0 >> 6);
               } else {
-                if (a0 < j.a_ext) tma_load_2d_pair(dA, j.mA, fb, a0, k);
-                if (a0 + 64 < j.a_ext) tma_load_2d_pair(dA + kBox, j.mA, fb, a0 + 64, k);
+                if (a0 < j.a_ext) tma_load_2d_pair(dAs, j.mA, fb, a0, k);
+                if (a0 + 64 < j.a_ext) tma_load_2d_pair(dAs + kBox, j.mA, fb, a0 + 64, k);
               }
               if (!j.b_mn) {
-                if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, k, b0);
+                if (!j.bk3 && b0 < j.b_ext) tma_load_2d_pair(dBs, j.mB, fb, k, b0);
               } else if (j.b3) {
-                if (b0 < j.b_ext) tma_load_3d_pair(dB, j.mB, fb, 0, j.bk0 + k, b0 >> 6);
+                if (b0 < j.b_ext) tma_load_3d_pair(dBs, j.mB, fb, 0, j.bk0 + k, b0 >> 6);
               } else {
-                if (b0 < j.b_ext) tma_load_2d_pair(dB, j.mB, fb, b0, j.bk0 + k);
-                if (b0 + 64 < j.b_ext) tma_load_2d_pair(dB + kBox, j.mB, fb, b0 + 64, j.bk0 + k);
+                if (b0 < j.b_ext) tma_load_2d_pair(dBs, j.mB, fb, b0, j.bk0 + k);
+                if (b0 + 64 < j.b_ext) tma_load_2d_pair(dBs + kBox, j.mB, fb, b0 + 64, j.bk0 + k);
               }
             }
+            if (leader) mbar_arrive_expect_tx(full_bar(s), bytes);
             ++issued;
+            if (++s == kPStages) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
         }
       }
