@@ -330,11 +330,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long u = pair + static_cast<long long>(k) * npairs;
     return u < total ? u : -1;
   };
+  // A slot is rewritten by the leader's producer once every consumer has
+  // arrived on its "empty" barrier.  A consumer in the leader's own CTA orders
+  // its read of the slot with a CTA-scope release (the writer is in its CTA);
+  // a cluster-scope one held the MMA-issuing thread ~1.3k cycles per unit.
+  // The peer's consumers read the peer's copy and release at cluster scope.
   auto fetch_unit = [&](uint32_t k) -> long long {
     const int slot = k % kRing;
     if (!mbar_wait_cluster_bounded(sfull_bar(slot), (k / kRing) & 1u, abort_flag, err, lim)) return -1;
     const int v = static_cast<int>(ld_shared_u32(ring_addr + 4u * slot));
-    mbar_arrive_cluster(mapa_shared(sempty_bar(slot), 0));
+    if (leader) {
+      mbar_arrive(sempty_bar(slot));
+    } else {
+      mbar_arrive_cluster(mapa_shared(sempty_bar(slot), 0));
+    }
     return v;
   };
   // The leader's producer claims each unit one unit ahead of publishing it
@@ -345,9 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int slot = k % kRing;
     if (!mbar_wait_bounded(sempty_bar(slot), ((k / kRing) & 1u) ^ 1u, abort_flag, err, lim)) return -1;
     if (u >= total) u = -1;
-    st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 0), static_cast<uint32_t>(u));
+    // the own CTA's copy first, ordered at CTA scope (its MMA issuer waits for
+    // it), then the peer's copy at cluster scope
+    tmem_slot[4 + slot] = static_cast<uint32_t>(u);
+    mbar_arrive(sfull_bar(slot));
     st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 1), static_cast<uint32_t>(u));
-    mbar_arrive_cluster(mapa_shared(sfull_bar(slot), 0));
     mbar_arrive_cluster(mapa_shared(sfull_bar(slot), 1));
     return u;
   };
@@ -625,7 +636,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+        if (lane == 0) {  // to the leader's MMA issuer: CTA scope from its own CTA
+          if (leader) {
+            mbar_arrive(tempty_bar(acc));
+          } else {
+            mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+          }
+        }
         if constexpr (Mode == kModeBwd) {
           if (j.type == kUnitR && lane == 0) bulk_wait_all();  // dX tiles written
           epilogue_bar();  // every store of this CTA's half of the unit is done or issued
