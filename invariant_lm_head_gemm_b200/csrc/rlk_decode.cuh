@@ -226,6 +226,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
       tma_prefetch_desc(&P.hid_k);
       const int h0 = kPair ? static_cast<int>(rank & 1u) * NB : 0;  // first hidden row held here
       bool ok = true;
+      // stage slot and phase kept incrementally, and each stage's addresses
+      // worked out before the wait for its slot: the copies go out as soon as
+      // the slot is free
+      int s = 0;
+      uint32_t ph = 0;
       for (uint32_t k = 0; ok; ++k) {
         const long long u = unit_of(k);
         if (u < 0) break;
@@ -237,30 +242,31 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
         if (kPair) kb_bytes += (w0 + kBM < P.ep.V ? kDecABox : 0u) + b_box;
         for (int kb = 0; kb < P.KB; kb += kDecKPerStage) {
           const int nk = min(kDecKPerStage, P.KB - kb);  // K blocks in this stage
-          const int s = issued % S;
-          const uint32_t ph = (issued / S) & 1u;
+          const uint32_t dA = sA + s * kDecABytes, dB = sB + s * b_bytes;
+          const uint32_t fb = kPair ? mapa_shared(full_bar(s), lead) : full_bar(s);
+          const uint32_t tx = nk * kb_bytes;
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
             ok = false;
             break;
           }
           if constexpr (kPair) {
-            const uint32_t fb = mapa_shared(full_bar(s), lead);
-            if (is_lead) mbar_arrive_expect_tx(full_bar(s), nk * kb_bytes);
+            if (is_lead) mbar_arrive_expect_tx(full_bar(s), tx);
             for (int i = 0; i < nk; ++i) {
-              if (a_in)
-                tma_load_2d_pair(sA + s * kDecABytes + i * kDecABox, &P.w_k, fb, (kb + i) * kBK, w0);
-              tma_load_2d_pair(sB + s * b_bytes + i * b_box, &P.hid_k, fb, (kb + i) * kBK, h0);
+              if (a_in) tma_load_2d_pair(dA + i * kDecABox, &P.w_k, fb, (kb + i) * kBK, w0);
+              tma_load_2d_pair(dB + i * b_box, &P.hid_k, fb, (kb + i) * kBK, h0);
             }
           } else {
-            mbar_arrive_expect_tx(full_bar(s), nk * kb_bytes);
+            mbar_arrive_expect_tx(fb, tx);
             for (int i = 0; i < nk; ++i) {
-              if (a_in)
-                tma_load_2d(sA + s * kDecABytes + i * kDecABox, &P.w_k, full_bar(s),
-                            (kb + i) * kBK, w0);
-              tma_load_2d(sB + s * b_bytes + i * b_box, &P.hid_k, full_bar(s), (kb + i) * kBK, 0);
+              if (a_in) tma_load_2d(dA + i * kDecABox, &P.w_k, fb, (kb + i) * kBK, w0);
+              tma_load_2d(dB + i * b_box, &P.hid_k, fb, (kb + i) * kBK, 0);
             }
           }
           ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
     }
@@ -269,7 +275,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && is_lead) {
       const uint32_t idesc = idesc_bf16_f32(kPair ? 2 * kBM : kBM, N, false, false);
-      uint32_t it = 0;
+      int s = 0;  // stage slot and phase, kept incrementally
+      uint32_t ph = 0;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
         if (unit_of(k) < 0) break;
@@ -277,10 +284,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
         if (!mbar_wait_bounded(tempty_bar(acc), ((k >> 1) & 1u) ^ 1u, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MR;
-        for (int kb = 0; kb < P.KB; kb += kDecKPerStage, ++it) {
+        for (int kb = 0; kb < P.KB; kb += kDecKPerStage) {
           const int nk = min(kDecKPerStage, P.KB - kb);
-          const int s = it % S;
-          if (!mbar_wait_bounded(full_bar(s), (it / S) & 1u, abort_flag, err)) {
+          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
             ok = false;
             break;
           }
@@ -303,6 +309,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
             umma_commit_pair_mask(empty_bar(s), pair_mask);
           } else {
             umma_commit(empty_bar(s));
+          }
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
           }
         }
         if (ok) {
