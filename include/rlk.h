@@ -369,6 +369,23 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
                                           uint64_t wait_limit_ns, int stall,
                                           uint32_t* chunk_done, uint32_t seq, void* stream);
 
+/* Test hook of the short-batch forward's fail-closed path: rlk_linear_logp_fwd
+ * (same arguments, layouts and ownership) for 1 <= T <= 224 rows, the sizes
+ * that run the short-batch kernel, with more: wait_limit_ns bounds every wait
+ * of the kernel (1 ms .. 2 s; the production entry points use 2 s); stall != 0
+ * makes the first CTA of every cluster wait for a second arrival on its first
+ * accumulator's "full" barrier, which never comes, so that its epilogue, the
+ * chain of the other CTAs and the MMA issuer all run out their waits and
+ * unwind.  The call returns RLK_OK (the launches are enqueued); the results
+ * are not to be used; rlk_read_device_error then reports RLK_DEVERR_TIMEOUT,
+ * and later calls on the same workspace and stream behave as on a fresh one.
+ * T outside 1 .. 224 or a limit outside the range: RLK_ERR_INVALID_ARG. */
+rlk_status rlk_test_linear_logp_fwd_stall(const rlk_bf16* hidden, const rlk_bf16* W,
+                                          const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                          float temperature, float* logp, float* entropy,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          uint64_t wait_limit_ns, int stall, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* rlk_status_string(rlk_status status);
 

@@ -229,6 +229,32 @@ def rlk_test_linear_logp_bwd_stall(hidden, W, targets, temperature, lse, entropy
     return dHidden, dW
 
 
+_fwd_stall_fn = None
+
+
+def rlk_test_linear_logp_fwd_stall(hidden, W, targets, temperature, workspace, out, wait_limit_ns,
+                                   stall, stream=None):
+    """Test hook of the short-batch forward's fail-closed path (T <= 224): every
+    wait bounded by wait_limit_ns and, when stall is set, one accumulator that
+    never reports full (the device error word then reports
+    RLK_DEVERR_TIMEOUT)."""
+    global _fwd_stall_fn
+    if _fwd_stall_fn is None:
+        f = lib().rlk_test_linear_logp_fwd_stall
+        f.argtypes = [_P, _P, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _P,
+                      ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, _P]
+        f.restype = ctypes.c_int
+        _fwd_stall_fn = f
+    T, H = hidden.shape
+    V = W.shape[0]
+    logp, entropy, lse = out
+    _check(_fwd_stall_fn(_ptr(hidden), _ptr(W), _ptr(targets), T, H, V, float(temperature),
+                         _ptr(logp), _ptr(entropy), _ptr(lse), _ptr(workspace), workspace.numel(),
+                         int(wait_limit_ns), int(stall), _stream(stream)),
+           "rlk_test_linear_logp_fwd_stall")
+    return logp, entropy, lse
+
+
 def rlk_gemm_bf16_f32(A, B, a_mn_major=False, b_mn_major=False, stream=None, out=None,
                       workspace=None):
     """C = A' . B'^T through the tensor-core mainloop (self-check entry).

@@ -345,8 +345,11 @@ rlk_status enqueue_fwd_partials_short(const rlk_bf16* hidden, const rlk_bf16* W,
                                       const int64_t* targets, int64_t T, int64_t H, int64_t Vloc,
                                       int64_t v0, float temperature, float* part_m, float* part_s,
                                       float* part_b, int64_t ldp, float* ytgt, uint32_t* err,
-                                      cudaStream_t st) {
+                                      cudaStream_t st, uint64_t wait_limit_ns = kWaitLimitNs,
+                                      int stall = 0) {
   DecArgs a;
+  a.wait_limit_ns = wait_limit_ns;
+  a.stall = stall;
   a.N = dec_width(T);
   const bool pair = a.N >= kDecPairMinN;
   if (!map_kmajor(&a.w_k, W, H, Vloc, H, kBM) ||
@@ -546,6 +549,40 @@ rlk_status rlk_linear_logp_fwd(const rlk_bf16* hidden, const rlk_bf16* W, const 
   return RLK_OK;
 }
 
+// Test hook (declared in rlk.h): the short-batch forward with a chosen bound
+// on every wait and, with stall set, one wait that nothing satisfies.
+rlk_status rlk_test_linear_logp_fwd_stall(const rlk_bf16* hidden, const rlk_bf16* W,
+                                          const int64_t* targets, int64_t T, int64_t H, int64_t V,
+                                          float temperature, float* logp, float* entropy,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          uint64_t wait_limit_ns, int stall, void* stream) {
+  rlk_status s = check_sizes(T, H, V, temperature);
+  if (s != RLK_OK) return s;
+  if (T < 1 || T > kDecMaxT || wait_limit_ns < 1000000ull || wait_limit_ns > kWaitLimitNs)
+    return RLK_ERR_INVALID_ARG;
+  if (!hidden || !W || !targets || !logp || !entropy || !lse || !workspace)
+    return RLK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(workspace, 256) ||
+      !aligned(targets, 8) || !aligned(logp, 4) || !aligned(entropy, 4) || !aligned(lse, 4))
+    return RLK_ERR_MISALIGNED;
+  const Layout L = layout(T, H, V);
+  if (workspace_bytes < L.fwd_end) return RLK_ERR_WORKSPACE_TOO_SMALL;
+  int sms = 0;
+  if ((s = check_device(&sms)) != RLK_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  float* pm = reinterpret_cast<float*>(ws + L.pm);
+  float* ps = reinterpret_cast<float*>(ws + L.ps);
+  float* pb = reinterpret_cast<float*>(ws + L.pb);
+  float* yt = reinterpret_cast<float*>(ws + L.yt);
+  s = enqueue_fwd_partials_short(hidden, W, targets, T, H, V, 0, temperature, pm, ps, pb,
+                                 fwd_groups(V), yt, err, st, wait_limit_ns, stall != 0 ? 1 : 0);
+  if (s != RLK_OK) return s;
+  return enqueue_combine(pm, ps, pb, fwd_groups(V), yt, targets, T, V, logp, entropy, lse, err,
+                         st);
+}
+
 rlk_status rlk_linear_logp_bwd(const rlk_bf16* hidden, const rlk_bf16* W, const int64_t* targets,
                                int64_t T, int64_t H, int64_t V, float temperature,
                                const float* lse, const float* entropy, const float* dlogp,
@@ -698,6 +735,8 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
     // Each C element is the same K-ordered dot product as in the pair tiles,
     // so the results do not depend on which path a row count takes.
     DecArgs d;
+    d.wait_limit_ns = kWaitLimitNs;
+    d.stall = 0;
     d.N = dec_width(M);
     if (!map_kmajor(&d.w_k, B, K, N, K, kBM) ||
         !map_kmajor(&d.hid_k, A, K, M, K, d.N >= kDecPairMinN ? d.N / 2 : d.N))

@@ -103,6 +103,9 @@ struct DecArgs {
   int KB;             // H / 64
   int NG;             // vocab splits of this W
   int stages;
+  uint64_t wait_limit_ns;  // bound of every wait (kWaitLimitNs outside the test hook)
+  int stall;          // test hook: CTA 0 of each cluster waits for a second arrival on its
+                      // first accumulator's "full" barrier, which never comes
 };
 
 // Dynamic shared memory of the kernel for MMA width N and `stages` stages.
@@ -174,6 +177,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
   const long long nclusters = gridDim.x / kDecCluster;
   const long long total = P.NG;
   uint32_t* err = P.err;
+  const uint64_t lim = P.wait_limit_ns;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -183,7 +187,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
       mbar_init(empty_bar(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
+      mbar_init(tfull_bar(a), P.stall != 0 && a == 0 && rank == 0 ? 2 : 1);
       mbar_init(tempty_bar(a), kPair ? 8 : 4);  // one arrival per epilogue warp (of both CTAs)
       for (int blk = 0; blk < kDecMaxBlocks; ++blk) mbar_init(hfull_bar(a, blk), 32);
       mbar_init(hempty_bar(a), 32);
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
           const uint32_t dA = sA + s * kDecABytes, dB = sB + s * b_bytes;
           const uint32_t fb = kPair ? mapa_shared(full_bar(s), lead) : full_bar(s);
           const uint32_t tx = nk * kb_bytes;
-          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err)) {
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err, lim)) {
             ok = false;
             break;
           }
@@ -281,12 +285,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
       for (uint32_t k = 0; ok; ++k) {
         if (unit_of(k) < 0) break;
         const int acc = k & 1;
-        if (!mbar_wait_bounded(tempty_bar(acc), ((k >> 1) & 1u) ^ 1u, abort_flag, err)) break;
+        if (!mbar_wait_bounded(tempty_bar(acc), ((k >> 1) & 1u) ^ 1u, abort_flag, err, lim)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MR;
         for (int kb = 0; kb < P.KB; kb += kDecKPerStage) {
           const int nk = min(kDecKPerStage, P.KB - kb);
-          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err)) {
+          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, err, lim)) {
             ok = false;
             break;
           }
@@ -341,14 +345,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
     // waits of one lane, shared with the warp; then each lane acquires
     auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
       int ok = 0;
-      if (lane == 0) ok = mbar_wait_bounded_sleep(bar, parity, abort_flag, err) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait_bounded_sleep(bar, parity, abort_flag, err, lim) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok) mbar_try_wait(bar, parity);
       return ok != 0;
     };
     auto warp_wait_cluster = [&](uint32_t bar, uint32_t parity) -> bool {
       int ok = 0;
-      if (lane == 0) ok = mbar_wait_cluster_bounded_sleep(bar, parity, abort_flag, err) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait_cluster_bounded_sleep(bar, parity, abort_flag, err, lim) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (ok) mbar_try_wait_cluster(bar, parity);
       return ok != 0;

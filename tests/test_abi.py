@@ -244,3 +244,20 @@ def test_stall_hook_rejects_limits_outside_its_range(L):
     assert f(p, p, p, 0, 64, 100, 1.0, p, p, p, p, p, p, p, 1 << 20, 100_000_000, 1,
              None, 0, None) == INVALID                              # T = 0
     assert f(*args, 100_000_000, 1, p, 0, None) == INVALID         # words without seq
+
+
+def test_forward_stall_hook_checks_its_arguments_first(L):
+    """The short-batch forward's test hook rejects T outside 1 .. 224 and limits
+    outside 1 ms .. 2 s before anything touches the device: these pointers are
+    never dereferenced."""
+    f = L.rlk_test_linear_logp_fwd_stall
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [ctypes.c_float] + \
+        [ctypes.c_void_p] * 4 + [ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    p = 0x10000
+    ok_limit = 100_000_000
+    assert f(p, p, p, 4, 64, 100, 1.0, p, p, p, p, 1 << 20, 10, 1, None) == INVALID
+    assert f(p, p, p, 4, 64, 100, 1.0, p, p, p, p, 1 << 20, 3_000_000_000, 1, None) == INVALID
+    assert f(p, p, p, 0, 64, 100, 1.0, p, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID
+    assert f(p, p, p, 225, 64, 100, 1.0, p, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID
+    assert f(p, p, p, 4, 64, 100, 1.0, None, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID

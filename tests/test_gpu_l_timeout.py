@@ -75,3 +75,41 @@ def test_stalled_backward_reports_timeout_and_the_next_call_is_unaffected():
     for a, b in ((lp2, lp), (en2, en), (ls2, ls)):
         assert torch.equal(_bits(a), _bits(b))
 
+
+
+@pytest.mark.parametrize("T", [16, 128, 200])
+def test_stalled_short_batch_forward_reports_timeout_and_the_next_call_is_unaffected(T):
+    """The short-batch forward (single-CTA MMA form at T = 16, CTA-pair form at
+    T = 128 and 200) with the first CTA of every cluster waiting for an
+    accumulator that never reports full: its epilogue, the chain of the other
+    three CTAs and the MMA issuer run out their 100 ms waits, the call returns,
+    the error word says timeout, and the next calls on the same workspace give
+    the results of a fresh one bit for bit."""
+    tau = 1.0
+    case = gu.random_case(T, 256, 20000, tau, seed=T + 77)
+    hid, W = gu.dev_bf16(case.hidden), gu.dev_bf16(case.W)
+    tg = gu.dev(case.targets, torch.int64)
+    ws = binding.make_workspace(T, 256, 20000, False)
+    ref = [t.clone() for t in binding.rlk_linear_logp_fwd(hid, W, tg, tau, ws)]
+    torch.cuda.synchronize()
+    assert binding.rlk_read_device_error(ws) == 0
+    out = tuple(torch.empty(T, device="cuda") for _ in range(3))
+    # the short bound alone changes nothing
+    binding.rlk_test_linear_logp_fwd_stall(hid, W, tg, tau, ws, out, LIMIT_NS, 0)
+    torch.cuda.synchronize()
+    assert binding.rlk_read_device_error(ws) == 0
+    for a, b in zip(out, ref):
+        assert torch.equal(_bits(a), _bits(b))
+    t0 = time.perf_counter()
+    binding.rlk_test_linear_logp_fwd_stall(hid, W, tg, tau, ws, out, LIMIT_NS, 1)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    flags = binding.rlk_read_device_error(ws)
+    assert flags & binding.RLK_DEVERR_TIMEOUT, flags
+    assert elapsed < 5.0, elapsed   # a few 100 ms bounds in a chain, not the 2 s default
+    for _ in range(2):
+        again = binding.rlk_linear_logp_fwd(hid, W, tg, tau, ws)
+        torch.cuda.synchronize()
+        assert binding.rlk_read_device_error(ws) == 0
+        for a, b in zip(again, ref):
+            assert torch.equal(_bits(a), _bits(b))
