@@ -330,13 +330,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long u = pair + static_cast<long long>(k) * npairs;
     return u < total ? u : -1;
   };
+  // The peer's copy of a slot completes the peer's "full" barrier by the
+  // store's own transaction count; the leader's copy by a CTA-scope arrival.
   // A slot is rewritten by the leader's producer once every consumer has
   // arrived on its "empty" barrier.  A consumer in the leader's own CTA orders
   // its read of the slot with a CTA-scope release (the writer is in its CTA);
   // a cluster-scope one held the MMA-issuing thread ~1.3k cycles per unit.
   // The peer's consumers read the peer's copy and release at cluster scope.
-  auto fetch_unit = [&](uint32_t k) -> long long {
+  auto fetch_unit = [&](uint32_t k, bool arm = false) -> long long {
     const int slot = k % kRing;
+    // the peer's producer arms its own copy's barrier for the leader's 4-byte
+    // asynchronous store (the phase completes once both have happened)
+    if (arm) mbar_arrive_expect_tx(sfull_bar(slot), 4u);
     if (!mbar_wait_cluster_bounded(sfull_bar(slot), (k / kRing) & 1u, abort_flag, err, lim)) return -1;
     const int v = static_cast<int>(ld_shared_u32(ring_addr + 4u * slot));
     if (leader) {
@@ -355,11 +360,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!mbar_wait_bounded(sempty_bar(slot), ((k / kRing) & 1u) ^ 1u, abort_flag, err, lim)) return -1;
     if (u >= total) u = -1;
     // the own CTA's copy first, ordered at CTA scope (its MMA issuer waits for
-    // it), then the peer's copy at cluster scope
+    // it); the peer's copy by an asynchronous store that completes the peer's
+    // barrier itself: a cluster-scope release here waited for this thread's
+    // copies still in flight (~1.3k cycles per unit)
     tmem_slot[4 + slot] = static_cast<uint32_t>(u);
     mbar_arrive(sfull_bar(slot));
-    st_shared_cluster_u32(mapa_shared(ring_addr + 4u * slot, 1), static_cast<uint32_t>(u));
-    mbar_arrive_cluster(mapa_shared(sfull_bar(slot), 1));
+    st_async_cluster_u32(mapa_shared(ring_addr + 4u * slot, 1), static_cast<uint32_t>(u),
+                         mapa_shared(sfull_bar(slot), 1));
     return u;
   };
 
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             u = publish_unit(k, claimed);
             if (u >= 0) claimed = atomicAdd(P.next_unit, 1u);
           } else {
-            u = fetch_unit(k);
+            u = fetch_unit(k, true);
           }
         } else {
           u = static_unit(k);

@@ -500,6 +500,17 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded_sleep(uint32_t bar, ui
   }
 }
 
+// Stores a 32-bit value into another CTA's shared memory without a release:
+// the store completes 4 bytes of the transaction count of that CTA's mbarrier
+// `cluster_bar`, whose phase then makes the value visible to its waiters.
+__device__ __forceinline__ void st_async_cluster_u32(uint32_t cluster_addr, uint32_t v,
+                                                     uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                   cluster_addr),
+               "r"(v), "r"(cluster_bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
