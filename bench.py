@@ -447,8 +447,9 @@ def run_ours(args):
     # through enough copies of x and W to exceed L2 (so W streams from HBM as
     # it would in a model), replayed 5 times.  Bound per shape: the larger of
     # the tensor time (2TNK at the burst peak) and the HBM time (x, W and y).
-    gemm = {"kernel": "T <= 224: decode_fwd_kernel store mode (operands swapped, 128 W rows per "
-                      "CTA); larger T: pair_kernel<kModeGemm> (256 x 256 pair tiles); fp32 out",
+    gemm = {"kernel": "T <= 224: decode_fwd_kernel store mode (operands swapped; 64 W rows per "
+                      "CTA for T <= 128 and N <= 8192, else 128); larger T: "
+                      "pair_kernel<kModeGemm> (256 x 256 pair tiles); fp32 out",
             "timing": "CUDA graph of 20 calls over rotating copies (> L2), replayed 5 times",
             "shapes": [], "us_per_call": [], "tflops": [], "gbs": [], "bound": [], "frac": []}
     for (gN, gK, gT) in ((512, 384, 70), (2048, 1024, 257), (5120, 5120, 33)):

@@ -283,8 +283,10 @@ rlk_status rlk_transition_logp(const float* x, const float* v, const float* prev
  * M, N, K >= 1; K and N multiples of 8, and M too when a_mn_major.  Needs a
  * workspace of rlk_gemm_workspace_bytes() bytes for its error word.  With
  * row-major A and B and M <= 224 it runs the short-batch forward kernel's
- * mainloop (operands swapped) with a plain store; every element is the same
- * K-ordered dot product either way, so C's bits do not depend on M. */
+ * mainloop (operands swapped) with a plain store, for M <= 128 and N <= 8192
+ * in a half-height form (64 rows of B per CTA on twice the CTAs);
+ * every element is the same K-ordered dot product on every path, so C's bits
+ * do not depend on M. */
 size_t rlk_gemm_workspace_bytes(void);
 rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, int64_t N,
                              int64_t K, int a_mn_major, int b_mn_major, float* C,

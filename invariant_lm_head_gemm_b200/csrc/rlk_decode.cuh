@@ -25,7 +25,14 @@
 //
 // A second epilogue (kStore) turns the kernel into the short-row path of the
 // plain dense GEMM: no fold and no chain, each accumulator column is stored
-// as C[t][n] (coalesced across the lanes of a warp).
+// as C[t][n] (coalesced across the lanes of a warp).  For a narrow C (few
+// W rows) the store path also has a half-height form (kHalf: single-CTA
+// MMA with M = 64, 64 W rows per CTA), which spreads the same W over twice
+// the CTAs.  It gains only 2-5%: a short GEMM's time follows K, not its
+// bytes or its CTA count (about 7 us plus 0.42 us per 128-wide K stage at
+// N = 512-8192 and 16-128 CTAs), i.e. each CTA's serial chain of 16-wide MMA
+// steps sets it.  An M = 64 accumulator fills TMEM lanes 0-15 of each warp's
+// lane quarter (rows 16q .. 16q+15 in quarter q).
 //
 // Numerics are those of the pair kernel, bit for bit:
 //  * each logit is the same bf16 dot product over H in the same 64-wide K
@@ -77,6 +84,8 @@ constexpr int kDecSplit = kDecCluster * kBM;
 constexpr int kDecKPerStage = 2;   // K blocks per pipeline stage
 constexpr uint32_t kDecABox = kBM * kBK * 2;                    // one 128 x 64 W box
 constexpr uint32_t kDecABytes = kDecKPerStage * kDecABox;       // a stage's W boxes
+constexpr int kDecHalfRows = kBM / 2;  // W rows per CTA of the half-height store form
+constexpr int kDecHalfMaxN = 128;      // largest N of the half-height form
 // full, empty per stage; tfull, tempty per accumulator; hfull per (hand
 // buffer, block), hempty per hand buffer; pfull, pempty per warp link; xfull,
 // xfree of the one-block epilogue; drain
@@ -109,26 +118,33 @@ struct DecArgs {
                       // first accumulator's "full" barrier, which never comes
 };
 
-// Dynamic shared memory of the kernel for MMA width N and `stages` stages.
-__host__ __device__ constexpr uint32_t dec_smem_bytes(int N, int stages, bool pair) {
+// Dynamic shared memory of the kernel for MMA width N and `stages` stages
+// (`half`: the half-height store form, whose W boxes hold 64 rows).
+__host__ __device__ constexpr uint32_t dec_smem_bytes(int N, int stages, bool pair, bool half = false) {
   return 1024u +
          static_cast<uint32_t>(stages) *
-             (kDecABytes + static_cast<uint32_t>(pair ? N / 2 : N) * kBK * 2u * kDecKPerStage) +
+             ((half ? kDecABytes / 2u : kDecABytes) +
+              static_cast<uint32_t>(pair ? N / 2 : N) * kBK * 2u * kDecKPerStage) +
          kDecEpiFloats * 4u + 2u * 3u * static_cast<uint32_t>(pair ? kDecMaxRows : kDecSingleMaxN) * 4u +
          kDecNumBars * 8u + 32u;
 }
 
 // The stage count the launcher takes for MMA width N: the most, at most
 // kDecMaxStages, whose plan fits in `limit` bytes; 0 if two stages do not fit.
-__host__ __device__ constexpr int dec_stages(int N, bool pair, uint32_t limit) {
+__host__ __device__ constexpr int dec_stages(int N, bool pair, uint32_t limit, bool half = false) {
   int S = kDecMaxStages;
-  while (S >= 2 && dec_smem_bytes(N, S, pair) > limit) --S;
+  while (S >= 2 && dec_smem_bytes(N, S, pair, half) > limit) --S;
   return S >= 2 ? S : 0;
 }
 
-template <bool kPair, bool kStore = false>
+template <bool kPair, bool kStore = false, bool kHalf = false>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid_constant__ DecArgs P) {
+  static_assert(!kHalf || (kStore && !kPair), "the half-height form is a single-CTA store form");
   constexpr int MR = DecForm<kPair>::kMaxRows;  // batch rows a hand buffer holds
+  constexpr int RB = kHalf ? kDecHalfRows : kBM;                  // W rows per CTA tile
+  constexpr uint32_t kABox = static_cast<uint32_t>(RB) * kBK * 2u;  // one RB x 64 W box
+  constexpr uint32_t kABytes = kDecKPerStage * kABox;
+  constexpr int kUnitRows = kDecCluster * RB;                     // W rows per unit
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -138,8 +154,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
   const uint32_t b_box = static_cast<uint32_t>(NB) * kBK * 2u;   // one NB x 64 hidden box
   const uint32_t b_bytes = kDecKPerStage * b_box;
   const uint32_t sA = smem_u32(smem);
-  const uint32_t sB = sA + S * kDecABytes;
-  float* XT = reinterpret_cast<float*>(smem + S * (kDecABytes + b_bytes));  // [4][32][kDecXStride]
+  const uint32_t sB = sA + S * kABytes;
+  float* XT = reinterpret_cast<float*>(smem + S * (kABytes + b_bytes));  // [4][32][kDecXStride]
   float* pass = XT + 4 * 32 * kDecXStride;           // [3][3][32] (m, s, b) from warp c to c+1
   float* hand = pass + 3 * 3 * 32;                   // [2][3][MR] incoming (m, s, b)
   uint64_t* bars = reinterpret_cast<uint64_t*>(hand + 2 * 3 * MR);
@@ -245,15 +261,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
       for (uint32_t k = 0; ok; ++k) {
         const long long u = unit_of(k);
         if (u < 0) break;
-        const int w0 = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM;
+        const int w0 = static_cast<int>(u) * kUnitRows + static_cast<int>(rank) * RB;
         const bool a_in = w0 < P.ep.V;  // a tile wholly past V is masked anyway: skip its loads
         // bytes one K block delivers to the full barrier (both CTAs' in the pair form;
         // the odd CTA's W tile starts kBM rows after the even one's)
-        uint32_t kb_bytes = (a_in ? kDecABox : 0u) + b_box;
-        if (kPair) kb_bytes += (w0 + kBM < P.ep.V ? kDecABox : 0u) + b_box;
+        uint32_t kb_bytes = (a_in ? kABox : 0u) + b_box;
+        if (kPair) kb_bytes += (w0 + kBM < P.ep.V ? kABox : 0u) + b_box;
         for (int kb = 0; kb < P.KB; kb += kDecKPerStage) {
           const int nk = min(kDecKPerStage, P.KB - kb);  // K blocks in this stage
-          const uint32_t dA = sA + s * kDecABytes, dB = sB + s * b_bytes;
+          const uint32_t dA = sA + s * kABytes, dB = sB + s * b_bytes;
           const uint32_t fb = kPair ? mapa_shared(full_bar(s), lead) : full_bar(s);
           const uint32_t tx = nk * kb_bytes;
           if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, err, lim)) {
@@ -263,13 +279,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
           if constexpr (kPair) {
             if (is_lead) mbar_arrive_expect_tx(full_bar(s), tx);
             for (int i = 0; i < nk; ++i) {
-              if (a_in) tma_load_2d_pair(dA + i * kDecABox, &P.w_k, fb, (kb + i) * kBK, w0);
+              if (a_in) tma_load_2d_pair(dA + i * kABox, &P.w_k, fb, (kb + i) * kBK, w0);
               tma_load_2d_pair(dB + i * b_box, &P.hid_k, fb, (kb + i) * kBK, h0);
             }
           } else {
             mbar_arrive_expect_tx(fb, tx);
             for (int i = 0; i < nk; ++i) {
-              if (a_in) tma_load_2d(dA + i * kDecABox, &P.w_k, fb, (kb + i) * kBK, w0);
+              if (a_in) tma_load_2d(dA + i * kABox, &P.w_k, fb, (kb + i) * kBK, w0);
               tma_load_2d(dB + i * b_box, &P.hid_k, fb, (kb + i) * kBK, 0);
             }
           }
@@ -285,7 +301,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && is_lead) {
-      const uint32_t idesc = idesc_bf16_f32(kPair ? 2 * kBM : kBM, N, false, false);
+      const uint32_t idesc = idesc_bf16_f32(kPair ? 2 * kBM : RB, N, false, false);
       int s = 0;  // stage slot and phase, kept incrementally
       uint32_t ph = 0;
       bool ok = true;
@@ -302,11 +318,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
             break;
           }
           tc_fence_after();
-          const uint32_t a_s = sA + s * kDecABytes, b_s = sB + s * b_bytes;
+          const uint32_t a_s = sA + s * kABytes, b_s = sB + s * b_bytes;
           for (int i = 0; i < nk; ++i) {
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(a_s + i * kDecABox + kk * 32u, 16u, 1024u);
+              const uint64_t ad = smem_desc_sw128(a_s + i * kABox + kk * 32u, 16u, 1024u);
               const uint64_t bd = smem_desc_sw128(b_s + i * b_box + kk * 32u, 16u, 1024u);
               const uint32_t accum = ((kb + i) | kk) != 0 ? 1u : 0u;
               if constexpr (kPair) {
@@ -369,15 +385,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
     if constexpr (kStore) {
       // The plain GEMM (C[T, V] = hidden . W^T, fp32): lane l of warp q holds
       // output column n = tile row 32q + l for the accumulator's batch rows;
-      // each row t is stored as one coalesced 128-byte run of the warp.
+      // each row t is stored as one coalesced 128-byte run of the warp.  In
+      // the half-height form lanes 0-15 of warp q hold tile rows 16q + l
+      // (64-byte runs) and lanes 16-31 read lanes no MMA wrote, which are
+      // not stored.
       float* C = P.ep.part_m;
+      const bool lane_row = !kHalf || lane < 16;
       for (uint32_t k = 0; ok; ++k) {
         const long long u = unit_of(k);
         if (u < 0) break;
         const int acc = k & 1;
         if (!warp_wait(tfull_bar(acc), (k >> 1) & 1u)) break;
         tc_fence_after();
-        const int n = static_cast<int>(u) * kDecSplit + static_cast<int>(rank) * kBM + q * 32 + lane;
+        const int n = static_cast<int>(u) * kUnitRows + static_cast<int>(rank) * RB +
+                      (kHalf ? q * 16 : q * 32) + lane;
         for (int blk = 0; blk < nblk; ++blk) {
           uint32_t r[32];
           const int cols = N == 16 ? 16 : 32;
@@ -400,7 +421,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_fwd_kernel(const __grid
               }
             }
           }
-          if (n < P.ep.V) {
+          if (lane_row && n < P.ep.V) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int t = blk * 32 + j;

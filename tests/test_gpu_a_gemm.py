@@ -50,11 +50,13 @@ def test_gemm_repeatable():
         assert torch.equal(C0, C1)
 
 
-@pytest.mark.parametrize("N,K", [(264, 136), (520, 4096), (8, 8), (5120, 640)])
+@pytest.mark.parametrize("N,K", [(264, 136), (520, 4096), (8, 8), (5120, 640), (8448, 64)])
 def test_short_row_counts_equal_rows_of_a_long_gemm(N, K):
     """GEMMs of at most 224 rows (row-major operands) run the short-batch kernel
     with the operands swapped and a plain store epilogue; every row must equal
-    that row of a 300-row GEMM, which runs the pair tiles, bit for bit."""
+    that row of a 300-row GEMM, which runs the pair tiles, bit for bit.  Up to
+    128 rows and 8192 columns that is the half-height (M = 64) form; N = 8448
+    and the counts above 128 take the 128-row forms."""
     g = torch.Generator().manual_seed(N + K)
     A = torch.randn(300, K, generator=g).to(torch.bfloat16).cuda()
     B = torch.randn(N, K, generator=g).to(torch.bfloat16).cuda()

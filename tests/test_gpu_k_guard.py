@@ -228,10 +228,11 @@ def test_transition_step_writes_nothing_outside_its_buffers():
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 8, 8), (33, 520, 136), (224, 264, 4096), (225, 264, 136),
-                                   (70, 512, 384)])
+                                   (70, 512, 384), (128, 8192, 64), (100, 8200, 72)])
 def test_dense_gemm_writes_nothing_outside_its_output(M, N, K):
-    """The dense GEMM's two paths (the short-batch kernel's store mode up to 224
-    rows, the pair tiles above) with ragged M, N and K: C and the workspace
+    """The dense GEMM's paths (the short-batch kernel's store mode up to 224
+    rows, in its half-height form up to 128 rows and 8192 columns; the pair
+    tiles above) with ragged M, N and K: C and the workspace
     guarded, C equal to the same call on plain allocations bit for bit and to
     an fp64 matmul within 1e-5."""
     g = torch.Generator().manual_seed(M + N + K)
