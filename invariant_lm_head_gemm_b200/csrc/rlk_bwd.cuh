@@ -153,22 +153,27 @@ __host__ __device__ inline BwdUnit bwd_seg_R(const BwdPlan& P, int c, int i) {
 // the row block varies fastest, then the column block.  The units in flight
 // then share a few W column blocks and a few dX row blocks, so neither the
 // chunk's W columns nor its dX rows have to stream from DRAM many times.
+// Odd groups take the column blocks in descending order, so a group starts on
+// the W columns the previous group's last units are still reading.
 constexpr int kHGroup = 8;
 
 __host__ __device__ inline BwdUnit bwd_seg_H(const BwdPlan& P, int c, int i) {
   const int full = P.MT / kHGroup;
   const int per_group = kHGroup * P.NH;
-  int m, n;
+  int g, m, n;
   if (i < full * per_group) {
-    const int g = i / per_group, r = i % per_group;
+    g = i / per_group;
+    const int r = i % per_group;
     n = r / kHGroup;
     m = g * kHGroup + r % kHGroup;
   } else {
     const int rem = P.MT % kHGroup;
     const int r = i - full * per_group;
+    g = full;
     n = r / rem;
     m = full * kHGroup + r % rem;
   }
+  if (g & 1) n = P.NH - 1 - n;
   return BwdUnit{kUnitH, c, m, n};
 }
 __host__ __device__ inline BwdUnit bwd_seg_D(const BwdPlan& P, int c, int i) {
