@@ -146,8 +146,13 @@ __host__ inline long long bwd_total_units(const BwdPlan& P) {
   return t;
 }
 
+// Recompute units: the row block varies fastest, in descending order on odd
+// vocab tiles (serpentine), so a tile's first units reuse the hidden rows the
+// previous tile's last units have just read.
 __host__ __device__ inline BwdUnit bwd_seg_R(const BwdPlan& P, int c, int i) {
-  return BwdUnit{kUnitR, c, i % P.MT, i / P.MT};
+  const int j = i / P.MT;
+  const int m = (j & 1) ? P.MT - 1 - i % P.MT : i % P.MT;
+  return BwdUnit{kUnitR, c, m, j};
 }
 // dHidden units of one chunk in groups of kHGroup row blocks: inside a group
 // the row block varies fastest, then the column block.  The units in flight
@@ -176,8 +181,12 @@ __host__ __device__ inline BwdUnit bwd_seg_H(const BwdPlan& P, int c, int i) {
   if (g & 1) n = P.NH - 1 - n;
   return BwdUnit{kUnitH, c, m, n};
 }
+// dW units: the column block varies fastest, in descending order on odd
+// vocab blocks (serpentine, for the same reuse of hidden's columns).
 __host__ __device__ inline BwdUnit bwd_seg_D(const BwdPlan& P, int c, int i) {
-  return BwdUnit{kUnitD, c, i / P.NH, i % P.NH};
+  const int v = i / P.NH;
+  const int n = (v & 1) ? P.NH - 1 - i % P.NH : i % P.NH;
+  return BwdUnit{kUnitD, c, v, n};
 }
 
 // Unit r of group g: H(g), then D(g), then R(g + 2).
