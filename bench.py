@@ -395,7 +395,7 @@ def run_ours(args):
     dec_us = [decode_us(Td) for Td in decode_rows]
     dec_gbs = [(V * H * 2 + Td * (H * 2 + 8 + 12)) / (u * 1e-6) / 1e9
                for Td, (u, _) in zip(decode_rows, dec_us)]
-    decode = {"kernel": "decode_fwd_kernel (T <= 224: operands swapped, 128 vocab rows per CTA, "
+    decode = {"kernel": "decode_fwd_kernel (T <= 256: operands swapped, 128 vocab rows per CTA, "
                         "N = T padded to 16/32; single-CTA MMA for N <= 32, CTA-pair MMA "
                         "(M = 256) from N = 64) + combine; larger T: the pair kernel",
               "bound": "hbm", "unit": "GB/s", "timing": "CUDA-graph replay, 20 calls",

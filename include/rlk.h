@@ -372,7 +372,7 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
                                           uint32_t* chunk_done, uint32_t seq, void* stream);
 
 /* Test hook of the short-batch forward's fail-closed path: rlk_linear_logp_fwd
- * (same arguments, layouts and ownership) for 1 <= T <= 224 rows, the sizes
+ * (same arguments, layouts and ownership) for 1 <= T <= 256 rows, the sizes
  * that run the short-batch kernel, with more: wait_limit_ns bounds every wait
  * of the kernel (1 ms .. 2 s; the production entry points use 2 s); stall != 0
  * makes the first CTA of every cluster wait for a second arrival on its first
@@ -381,7 +381,7 @@ rlk_status rlk_test_linear_logp_bwd_stall(const rlk_bf16* hidden, const rlk_bf16
  * unwind.  The call returns RLK_OK (the launches are enqueued); the results
  * are not to be used; rlk_read_device_error then reports RLK_DEVERR_TIMEOUT,
  * and later calls on the same workspace and stream behave as on a fresh one.
- * T outside 1 .. 224 or a limit outside the range: RLK_ERR_INVALID_ARG. */
+ * T outside 1 .. 256 or a limit outside the range: RLK_ERR_INVALID_ARG. */
 rlk_status rlk_test_linear_logp_fwd_stall(const rlk_bf16* hidden, const rlk_bf16* W,
                                           const int64_t* targets, int64_t T, int64_t H, int64_t V,
                                           float temperature, float* logp, float* entropy,

@@ -234,7 +234,7 @@ _fwd_stall_fn = None
 
 def rlk_test_linear_logp_fwd_stall(hidden, W, targets, temperature, workspace, out, wait_limit_ns,
                                    stall, stream=None):
-    """Test hook of the short-batch forward's fail-closed path (T <= 224): every
+    """Test hook of the short-batch forward's fail-closed path (T <= 256): every
     wait bounded by wait_limit_ns and, when stall is set, one accumulator that
     never reports full (the device error word then reports
     RLK_DEVERR_TIMEOUT)."""

@@ -734,7 +734,7 @@ rlk_status rlk_gemm_bf16_f32(const rlk_bf16* A, const rlk_bf16* B, int64_t M, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(workspace);
 
-  if (!a_mn_major && !b_mn_major && M <= kDecMaxT) {
+  if (!a_mn_major && !b_mn_major && M <= kDecGemmMaxM) {
     // Few rows: the short-batch kernel with the operands swapped (B's rows on
     // the MMA's M side, A's M rows on its N side) and a plain store epilogue.
     // Each C element is the same K-ordered dot product as in the pair tiles,

@@ -1,4 +1,4 @@
-// rlk_decode.cuh -- forward for short batches (rollout / decode shapes, T <= 224
+// rlk_decode.cuh -- forward for short batches (rollout / decode shapes, T <= 256
 // rows): the same per-split triples as the pair kernel's forward, produced
 // with the operands swapped so that the tensor cores do not pad T up to 256.
 //
@@ -20,7 +20,7 @@
 //    rows but only half of the N hidden rows (B is split along N across the
 //    pair), and each CTA's TMEM receives its 128 W rows x all N columns, so
 //    the epilogue is the same.  Halving the hidden bytes per CTA lets N reach
-//    224 (three stages) where the single form would hold 56 KB of hidden per
+//    256 (three stages) where the single form would hold 64 KB of hidden per
 //    stage, and gives N = 128 four stages instead of three.
 //
 // A second epilogue (kStore) turns the kernel into the short-row path of the
@@ -68,8 +68,10 @@
 namespace rlk {
 
 constexpr int kDecMaxRows = 256;    // largest N of the pair form (hand buffer rows)
-constexpr int kDecMaxT = 224;       // largest T the launcher sends here: at N = 256 a stage
-                                    // holds as much hidden as W and the pair kernel is faster
+constexpr int kDecMaxT = 256;       // largest T the forward sends here (one 256-row tile of
+                                    // the pair kernel, whose 297 splits on 74 pairs take five
+                                    // rounds, the last with one unit; here nine on 33 clusters)
+constexpr int kDecGemmMaxM = 224;   // largest M of the plain GEMM's short path (store mode)
 constexpr int kDecSingleMaxN = 128; // largest N of the single form
 constexpr int kDecPairMinN = 64;    // N from which the pair form is launched
 constexpr int kDecCluster = 4;      // CTAs per vocab split

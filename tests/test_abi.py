@@ -247,7 +247,7 @@ def test_stall_hook_rejects_limits_outside_its_range(L):
 
 
 def test_forward_stall_hook_checks_its_arguments_first(L):
-    """The short-batch forward's test hook rejects T outside 1 .. 224 and limits
+    """The short-batch forward's test hook rejects T outside 1 .. 256 and limits
     outside 1 ms .. 2 s before anything touches the device: these pointers are
     never dereferenced."""
     f = L.rlk_test_linear_logp_fwd_stall
@@ -259,5 +259,5 @@ def test_forward_stall_hook_checks_its_arguments_first(L):
     assert f(p, p, p, 4, 64, 100, 1.0, p, p, p, p, 1 << 20, 10, 1, None) == INVALID
     assert f(p, p, p, 4, 64, 100, 1.0, p, p, p, p, 1 << 20, 3_000_000_000, 1, None) == INVALID
     assert f(p, p, p, 0, 64, 100, 1.0, p, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID
-    assert f(p, p, p, 225, 64, 100, 1.0, p, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID
+    assert f(p, p, p, 257, 64, 100, 1.0, p, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID
     assert f(p, p, p, 4, 64, 100, 1.0, None, p, p, p, 1 << 20, ok_limit, 1, None) == INVALID

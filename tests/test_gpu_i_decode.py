@@ -1,4 +1,4 @@
-"""Short batches (rollout / decode shapes, T <= 224) run the forward with the
+"""Short batches (rollout / decode shapes, T <= 256) run the forward with the
 operands swapped (decode_fwd_kernel): 128 vocab rows per CTA, N = T rounded
 up to 32, in the single-CTA MMA form up to N = 32 and the CTA-pair form
 (M = 256, each CTA holding half of the N hidden rows) from N = 64.  Its logp, entropy and lse must be the pair kernel's bit for
@@ -18,7 +18,7 @@ from tests import gpu_util as gu
 pytestmark = pytest.mark.gpu
 
 SHORT_T = [1, 2, 3, 4, 15, 16, 17, 31, 32, 33, 63, 64, 65, 96, 100, 127, 128, 129, 160, 161,
-           200, 224, 225, 256]
+           200, 224, 225, 240, 255, 256]
 
 
 def _bits(a):
@@ -27,7 +27,7 @@ def _bits(a):
 
 @pytest.mark.parametrize("H,V,tau", [(1024, 151936, 0.7), (256, 20000, 1.0), (64, 1000, 1.3)])
 def test_short_batches_equal_rows_of_a_long_batch(H, V, tau):
-    base_T = 300                                   # > 224: the pair kernel
+    base_T = 300                                   # > 256: the pair kernel
     case = gu.random_case(base_T, H, V, tau, seed=H + V)
     hid, W = gu.dev_bf16(case.hidden), gu.dev_bf16(case.W)
     tg = gu.dev(case.targets, torch.int64)
@@ -56,7 +56,8 @@ EDGE = [
     (32, 256, 3000, 1.0),  # the widest single-CTA form
     (33, 256, 3000, 1.0),  # the narrowest pair form: the odd CTA holds one valid row
     (200, 192, 2500, 0.8), # N = 224, ragged V
-    (224, 64, 5000, 0.9),  # the largest short batch
+    (224, 64, 5000, 0.9),  # N = 224
+    (256, 64, 5000, 0.9),  # the largest short batch, N = 256
     (129, 4096, 1537, 1.0),  # long K, N = 160
     (3, 4096, 1537, 1.0),  # long K, last split one tile and a column
 ]

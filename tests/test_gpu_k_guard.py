@@ -5,8 +5,9 @@ the calls every guard byte must be unchanged.  The kernels write past ragged
 edges with TMA stores and vector stores (dX boxes at T and at chunk tails, dW
 rows at V, the dHidden accumulator, split partials), so the shapes are ragged
 on purpose: T on both sides of the switch between the two short-batch MMA
-forms (32 / 33), of the short-batch switch (224 / 225) and of the 256-row
-tile (256 / 257), V on both sides of the 8192-row backward chunk, H at its
+forms (32 / 33), at the short-batch kernel's N = 224 / 256 (T = 224 / 225)
+and on both sides of the switch to the pair kernel's 256-row tiles (256 /
+257), V on both sides of the 8192-row backward chunk, H at its
 smallest and at the model's size.  The guarded results must also equal the
 results of the same calls on plain allocations bit for bit, and the fp64
 oracle within the parity tolerances (fail closed, zero mismatches: VIME

@@ -77,10 +77,10 @@ def test_stalled_backward_reports_timeout_and_the_next_call_is_unaffected():
 
 
 
-@pytest.mark.parametrize("T", [16, 128, 200])
+@pytest.mark.parametrize("T", [16, 128, 200, 256])
 def test_stalled_short_batch_forward_reports_timeout_and_the_next_call_is_unaffected(T):
     """The short-batch forward (single-CTA MMA form at T = 16, CTA-pair form at
-    T = 128 and 200) with the first CTA of every cluster waiting for an
+    T = 128, 200 and 256) with the first CTA of every cluster waiting for an
     accumulator that never reports full: its epilogue, the chain of the other
     three CTAs and the MMA issuer run out their 100 ms waits, the call returns,
     the error word says timeout, and the next calls on the same workspace give
